@@ -1,0 +1,423 @@
+"""Bench: quantized rows/s of the row-wise INT4 path on B200, with the lookup's GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload kaggle] [--impl reference]
+
+One step is one pass of the whole path over the workload: quantize every table
+(greedy search, FP16 scale/bias, packed codes), one sum-pooled embedding-bag call
+over the packed tables, and dequantization of every packed row. `value` is rows
+quantized per second of step time, all ranks together; the lookup's throughput
+is reported beside it in `embbag`.
+
+Multi-GPU (torchrun, one process per GPU): every rank quantizes an independent
+set of tables (the workload drawn with seed = rank), with no collective on the
+data path; timing is the max over ranks (weak scaling).
+
+--impl reference times the CPU oracle on the same workload (a bounded sample of
+rows per step, extrapolated to the whole step), on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from int4_row_wise_b200 import workloads as W  # noqa: E402
+
+METRIC = "quantized rows/s and INT4 embedding-bag GB/s (fraction of B200 HBM roofline)"
+FLOPS_PER_ELEMENT_EVAL = 10      # sub, div, rint, 2 clamps, mul, add, sub, mul, add
+EVALS_PER_ROW = 1 + 2 * 168      # initial clip + two candidates per move
+SM_COUNT_NOMINAL = 148
+FP32_LANES_PER_SM = 128
+# dram bytes read + written per quantized row, from the committed ncu capture of the
+# quantizer (profiles/quantize_rows_kernel_d16.md); valid only for the kernel source
+# whose sha256 prefix is recorded with it.
+NCU_QUANT_TRAFFIC = {"kernel_sha": None, "bytes_per_row": None}
+
+
+def _workload_desc(wl: W.Workload) -> str:
+    pool = wl.pooling[0] if wl.pooling[0] == wl.pooling[1] else f"U[{wl.pooling[0]},{wl.pooling[1]}]"
+    ids = "uniform" if wl.zipf_alpha is None else f"Zipf({wl.zipf_alpha})" + (" permuted" if wl.permute_ids else "")
+    return (f"{wl.name}: {wl.n_tables} fp32 tables, d={wl.d}, {wl.total_rows} rows ({wl.values}); "
+            f"embedding bag batch {wl.batch} x {wl.n_tables} tables, pooling {pool}, {ids} ids")
+
+
+def _config(wl: W.Workload, n_gpus: int) -> dict:
+    return {"workload": _workload_desc(wl), "tables": wl.n_tables, "d": wl.d, "rows_per_rank": wl.total_rows,
+            "batch": wl.batch, "pooling": list(wl.pooling), "seed": "rank", "parallelism": f"dp{n_gpus}",
+            "l2": "inputs larger than L2 (fp32 tables %.0f MB > 126 MB)" % (wl.total_rows * wl.d * 4 / 1e6)}
+
+
+def _kernel_sha() -> str:
+    p = os.path.join(ROOT, "int4_row_wise_b200", "csrc", "dq_quantize.cu")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def _unique_bag_bytes(wl: W.Workload, idx: np.ndarray, off: np.ndarray) -> int:
+    """Algorithmic bytes of one lookup call: unique packed rows touched per table,
+    the ids, the offsets and the output."""
+    rb = (wl.d + 1) // 2 + 4
+    B = wl.batch
+    uniq = 0
+    for t in range(wl.n_tables):
+        uniq += np.unique(idx[off[t * B]:off[(t + 1) * B]]).size
+    return uniq * rb + idx.nbytes + off.nbytes + B * wl.n_tables * wl.d * 4
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.sel = None
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(device_index)
+            self.sel = "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+        except Exception:
+            self.sel = None
+
+    def __enter__(self):
+        if self.sel is None:
+            return self
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out = ""
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in getattr(self, "lines", []):
+            f = [v.strip() for v in l.split(",")]
+            if len(f) < 8:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, f[4:8]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle as baseline
+# ---------------------------------------------------------------------------
+class OracleBench:
+    """Times the CPU oracle on bounded samples of a workload and extrapolates one
+    step (quantize + dequantize every row, one lookup call)."""
+
+    def __init__(self, wl: W.Workload):
+        import oracle
+        self.oracle = oracle
+        self.wl = wl
+        self.cores = len(os.sched_getaffinity(0))
+        big = int(np.argmax(wl.rows))
+        cal = W.table_rows(wl, big, 0, min(256, wl.rows[big]))
+        t0 = time.perf_counter()
+        oracle.quantize_rows(cal, nthreads=1)
+        self.per_row_core = (time.perf_counter() - t0) / cal.shape[0]
+        self.bag = W.lookup_batch(wl)
+        self.tabs = [W.random_packed_table(n, wl.d, 77 + t) for t, n in enumerate(wl.rows)]
+
+    def step(self, target_s: float, seed: int = 0):
+        """Returns (rows/s, seconds per step, sample description)."""
+        wl, oracle = self.wl, self.oracle
+        rng = np.random.default_rng(1234 + seed)
+        n_sample = int(max(self.cores * 16, min(wl.total_rows, target_s * self.cores / self.per_row_core * 0.8)))
+        share = np.array(wl.rows, dtype=np.float64) / wl.total_rows
+        per_table = np.minimum(np.maximum(1, np.round(share * n_sample).astype(np.int64)), np.array(wl.rows))
+        x = np.concatenate([W.sample_rows(wl, t, np.sort(rng.choice(wl.rows[t], int(k), replace=False)))
+                            for t, k in enumerate(per_table)])
+        t0 = time.perf_counter()
+        codes, sb, _, _ = oracle.quantize_rows(x, nthreads=self.cores)
+        tq = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.dequantize_rows(codes, sb, wl.d)
+        tdq = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        oracle.embbag(self.tabs, wl.d, self.bag[0], self.bag[1], wl.batch, nthreads=self.cores)
+        tbag = time.perf_counter() - t0
+        n = x.shape[0]
+        step_s = (tq + tdq) * wl.total_rows / n + tbag
+        sample = (f"{n} rows sampled across all {wl.n_tables} tables in proportion to their sizes "
+                  f"(quantize {tq:.2f} s + dequantize {tdq:.3f} s, scaled to {wl.total_rows} rows) "
+                  f"+ one full lookup call ({tbag:.3f} s)")
+        return wl.total_rows / step_s, step_s, sample
+
+
+def run_reference(args, wl: W.Workload) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    ob = OracleBench(wl)
+    per_step = max(1.0, args.ref_seconds * 10 / (args.warmup + args.steps))
+    steps, sample = [], ""
+    for i in range(args.warmup + args.steps):
+        rate, step_s, sample = ob.step(per_step, seed=i)
+        if i >= args.warmup:
+            steps.append(step_s)
+    step_s = float(np.mean(steps))
+    value = wl.total_rows / step_s
+    line = {"metric": METRIC, "value": value, "unit": "rows/s", "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(wl, 1),
+            "cpu_baseline": {"value": value, "unit": "rows/s", "cores": ob.cores, "kind": "oracle",
+                             "sample": f"per step: {sample}"},
+            "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the CUDA path
+# ---------------------------------------------------------------------------
+def run_gpu(args, wl: W.Workload) -> None:
+    import torch
+    import torch.distributed as dist
+
+    import int4_row_wise_b200 as dq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    dq.load()
+
+    # --- inputs, generated on the host (seeded per rank) and made resident in HBM
+    wlr = W.workload(wl.name, seed=rank)
+    host_tables = [W.table_rows(wlr, t) for t in range(wlr.n_tables)]
+    xs = [torch.from_numpy(h).to(dev) for h in host_tables]
+    d = wlr.d
+    cld = dq._codes_ld(d)
+    codes = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wlr.rows]
+    sbs = [torch.empty((n, 2), dtype=torch.int16, device=dev) for n in wlr.rows]
+    deq = [torch.empty((n, d), dtype=torch.float32, device=dev) for n in wlr.rows]
+    n_batches = 4
+    batches_h = [W.lookup_batch(wlr, batch_id=i) for i in range(n_batches)]
+    batches = [(torch.from_numpy(i).to(dev), torch.from_numpy(o).to(dev)) for i, o in batches_h]
+    bag_bytes = [_unique_bag_bytes(wlr, i, o) for i, o in batches_h]
+    out = torch.empty((wlr.batch, wlr.n_tables * d), dtype=torch.float32, device=dev)
+    tables = [dq.PackedTable(c, s) for c, s in zip(codes, sbs)]
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = sum(1 for n in wlr.rows if n > 0) * 2 + 1
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+
+    def step(k: int, timed: bool):
+        e = ev[k] if timed else None
+        if e:
+            e[0].record(stream)
+        for x, c, s in zip(xs, codes, sbs):
+            dq.dq_quantize_rows_int4(x, x.shape[0], d, d, c, cld, s, None, None, dq.DQ_MODE_GREEDY, None, stream)
+        if e:
+            e[1].record(stream)
+        bi, bo = batches[k % n_batches]
+        dq.dq_embbag_int4_fwd(tables, d, bi, bo, wlr.batch, out, None, stream)
+        if e:
+            e[2].record(stream)
+        for c, s, o in zip(codes, sbs, deq):
+            dq.dq_dequantize_rows(c, cld, s, c.shape[0], d, o, d, stream)
+        if e:
+            e[3].record(stream)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    for k in range(args.warmup):
+        step(k, False)
+    barrier()
+    sampler = ClockSampler(dev.index)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with sampler:
+        t_start.record(stream)
+        for k in range(args.steps):
+            step(k, True)
+        t_end.record(stream)
+        barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in ev)
+    bag_ms = sum(e[1].elapsed_time(e[2]) for e in ev)
+    dq_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
+    clocks = sampler.summary()
+
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    rows_all = wlr.total_rows * world * args.steps
+    value = rows_all / (total_ms / 1e3)
+
+    # --- roofline of the dominant kernel (the quantizer: FP32-ALU bound)
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+    peak_tflops = 2 * FP32_LANES_PER_SM * sms * 1965e6 / 1e12
+    q_flops = float(FLOPS_PER_ELEMENT_EVAL * EVALS_PER_ROW * d) * wlr.total_rows * args.steps
+    achieved = q_flops / (q_ms / 1e3) / 1e12
+    traffic = None
+    if NCU_QUANT_TRAFFIC["kernel_sha"] == _kernel_sha() and NCU_QUANT_TRAFFIC["bytes_per_row"]:
+        traffic = NCU_QUANT_TRAFFIC["bytes_per_row"] * wlr.total_rows / max(1, sum(1 for n in wlr.rows if n))
+
+    # --- the lookup's own throughput (unique algorithmic bytes per call)
+    bag_gbs = sum(bag_bytes[k % n_batches] for k in range(args.steps)) / (bag_ms / 1e3) / 1e9
+    hbm = _measured_hbm()
+
+    # --- end to end through the public API with pinned host buffers
+    e2e = run_e2e(args, wlr, host_tables, batches_h, dev, stream, dq) if rank == 0 else None
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ob = OracleBench(wlr)
+        rate, step_s, sample = ob.step(args.ref_seconds)
+        cpu = {"value": rate, "unit": "rows/s", "cores": ob.cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": _config(wlr, world),
+            "roofline": {"bound": "alu", "kernel": "quantize_rows_kernel", "achieved": achieved,
+                         "peak": peak_tflops, "unit": "TFLOP/s", "frac": achieved / peak_tflops,
+                         "traffic": traffic,
+                         "peak_source": f"2 x {FP32_LANES_PER_SM} FP32 lanes x {sms} SMs x 1965 MHz (FMA = 2 flops)",
+                         "work": f"{FLOPS_PER_ELEMENT_EVAL} flops x {EVALS_PER_ROW} evaluations x d per row"},
+            "embbag": {"value": bag_gbs, "unit": "GB/s", "peak": hbm, "frac": bag_gbs / hbm,
+                       "bytes_per_call": int(np.mean(bag_bytes)), "us_per_call": bag_ms / args.steps * 1e3,
+                       "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)"},
+            "phases_ms_per_step": {"quantize": q_ms / args.steps, "embbag": bag_ms / args.steps,
+                                   "dequantize": dq_ms / args.steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _measured_hbm() -> float:
+    try:
+        return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
+    except Exception:
+        return 6650.0  # fallback figure for this pool
+
+
+def run_e2e(args, wl, host_tables, batches_h, dev, stream, dq) -> dict:
+    """Same step through the public Python API, from and to pinned host memory:
+    H2D of the tables and the lookup batch, quantize, look up, dequantize, and D2H
+    of the packed tables, the pooled output and the dequantized rows."""
+    import torch
+    pin_x = [torch.from_numpy(h).pin_memory() for h in host_tables]
+    pin_b = [(torch.from_numpy(i).pin_memory(), torch.from_numpy(o).pin_memory()) for i, o in batches_h]
+    d = wl.d
+    cld = dq._codes_ld(d)
+    xs = [torch.empty_like(p, device=dev) for p in pin_x]
+    h_codes = [torch.empty((n, cld), dtype=torch.uint8).pin_memory() for n in wl.rows]
+    h_sb = [torch.empty((n, 2), dtype=torch.int16).pin_memory() for n in wl.rows]
+    h_deq = [torch.empty((n, d), dtype=torch.float32).pin_memory() for n in wl.rows]
+    h_out = torch.empty((wl.batch, wl.n_tables * d), dtype=torch.float32).pin_memory()
+    h2d = sum(p.numel() * 4 for p in pin_x) + pin_b[0][0].numel() * 4 + pin_b[0][1].numel() * 4
+    d2h = sum(c.numel() + s.numel() * 2 + q.numel() * 4 for c, s, q in zip(h_codes, h_sb, h_deq)) + h_out.numel() * 4
+
+    def step(k):
+        for p, x in zip(pin_x, xs):
+            x.copy_(p, non_blocking=True)
+        bi = pin_b[k % len(pin_b)][0].to(dev, non_blocking=True)
+        bo = pin_b[k % len(pin_b)][1].to(dev, non_blocking=True)
+        packed = []
+        for x, hc, hs in zip(xs, h_codes, h_sb):
+            c, s, _, _ = dq.quantize_rows(x, with_loss=False)
+            packed.append(dq.PackedTable(c, s))
+        out = dq.embbag(packed, d, bi, bo, wl.batch)
+        for (c, s), hc, hs, hq in zip(packed, h_codes, h_sb, h_deq):
+            hq.copy_(dq.dequantize_rows(c, s, d), non_blocking=True)
+            hc.copy_(c, non_blocking=True)
+            hs.copy_(s, non_blocking=True)
+        h_out.copy_(out, non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
+    for k in range(2):
+        step(k)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(steps):
+        step(k)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / steps
+    return {"value": wl.total_rows / (ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+
+
+def main(argv=None) -> None:
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="kaggle", choices=W.WORKLOADS)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--ref-seconds", type=float, default=12.0,
+                    help="seconds of oracle work in the CPU baseline (the reference arm spends ~10x this in all)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = W.workload(args.workload, seed=0)
+    if args.impl == "reference":
+        run_reference(args, wl)
+    else:
+        run_gpu(args, wl)
+
+
+if __name__ == "__main__":
+    main()

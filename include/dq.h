@@ -1,0 +1,163 @@
+/*
+ * dq.h -- C ABI of libdq: row-wise INT4 quantization of embedding tables and the
+ * sum-pooled INT4 embedding bag, as hand-written CUDA kernels for sm_100a (B200).
+ *
+ * The method: "Post-Training 4-bit Quantization on Embedding Tables" (Guan et al.,
+ * 2019), review page, section 提出的方法 (proposed method): each embedding row gets
+ * its own uniform 4-bit quantizer (bullet 1), with the clipping thresholds chosen
+ * by a greedy search that walks toward a local minimum of the squared error, and
+ * the scale and bias stored as FP16 (bullet 2; section 主要发现 / main findings,
+ * bullet 4: 13.28% of the FP32 size at d=128). The lookup: "Deep Learning
+ * Recommendation Model for Personalization and Recommendation Systems", section
+ * 提出的方法 (proposed method), bullet 1 (sparse ids mapped to dense vectors by
+ * embedding tables), summed over each bag of ids.
+ *
+ * Packed row format (shared by all entry points):
+ *   codes       d 4-bit codes, two per byte: byte m = q[2m] | q[2m+1] << 4; for odd d
+ *               the last byte's high nibble is 0. Row r starts at codes + r*codes_ld.
+ *   scale_bias  [n_rows][2] binary16 bit patterns {scale, bias}; element k of row r
+ *               decodes as fma(q_k, scale, bias) in binary32 (one rounding).
+ *
+ * Quantization of one row x[0..d-1] (binary32 throughout, round to nearest even):
+ *   xmin, xmax, R = xmax - xmin, step = R / 200; grid points lo(i) = fma(i, step, xmin),
+ *   hi(j) = fma(-j, step, xmax). L(lo, hi) is the squared reconstruction error with
+ *   s = (hi - lo) / 15, q = clamp(rint((x - lo) / s), 0, 15), xhat = fma(q, s, lo),
+ *   summed pairwise (recursive halving, padded with zeros to a power of two).
+ *   Starting from (0, 0), each of 168 moves (while the width exceeds 0.16 * R) tries
+ *   (i+1, j) and (i, j+1), moves to the lower loss (to (i+1, j) on a tie), and keeps
+ *   the first lowest loss seen. Then scale = fp16((hi* - lo*) / 15), bias = fp16(lo*),
+ *   q = clamp(rint((x - bias) / scale), 0, 15) with IEEE division (q = 0 when scale
+ *   is 0). DQ_MODE_MINMAX skips the moves (the plain min/max quantizer).
+ *
+ * Conventions for every entry point:
+ *   - All data pointers are DEVICE pointers (except `tables`, a host array). The
+ *     caller owns every buffer; the library allocates no memory and keeps no
+ *     state besides cached device attributes.
+ *   - Calls are asynchronous and stream-ordered on `cuda_stream` (a cudaStream_t;
+ *     NULL = the legacy default stream). Outputs are valid after the stream is
+ *     synchronized. Calls may be made from several host threads.
+ *   - Arguments are validated on the host before anything is enqueued:
+ *     DQ_ERR_INVALID_ARG, nothing launched. A failed launch returns DQ_ERR_CUDA.
+ *     dq_last_error() gives the calling thread's last detailed message.
+ *   - n_rows == 0 or batch == 0 is a no-op returning DQ_OK.
+ *   - Data errors are preconditions and are never trapped on the device. When
+ *     `d_flags` (a device uint32) is non-NULL the kernels OR DQ_FLAG_* bits into
+ *     it; read it after synchronizing. Out-of-range ids and decreasing offsets
+ *     are always skipped (contribute nothing), flagged or not.
+ */
+#ifndef DQ_H
+#define DQ_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum dq_status {
+    DQ_OK = 0,
+    DQ_ERR_INVALID_ARG = 1,  /* bad pointer, size, stride, mode or limit; nothing launched */
+    DQ_ERR_UNSUPPORTED = 2,  /* no sm_100-class device or no kernel for the request */
+    DQ_ERR_CUDA = 3          /* a CUDA runtime call or launch failed; see dq_last_error() */
+} dq_status;
+
+enum { DQ_MODE_GREEDY = 0, DQ_MODE_MINMAX = 1 };
+
+enum {
+    DQ_FLAG_BAD_INDEX = 1u,      /* an id < 0 or >= the table's n_rows was skipped */
+    DQ_FLAG_BAD_OFFSETS = 2u,    /* a bag with offsets[g+1] < offsets[g] was treated as empty */
+    DQ_FLAG_NONFINITE = 4u,      /* an input row held a NaN or an infinity */
+    DQ_FLAG_FP16_OVERFLOW = 8u   /* a row's scale or bias overflowed binary16 */
+};
+
+#define DQ_MAX_D 1024
+#define DQ_MAX_TABLES 64
+
+/* One packed table for the embedding bag. codes and scale_bias are device
+ * pointers in the packed row format above. */
+typedef struct dq_table {
+    const uint8_t *codes;
+    const uint16_t *scale_bias;
+    int64_t n_rows;
+    int64_t codes_ld;   /* bytes between rows, >= (d + 1) / 2 */
+} dq_table;
+
+/*
+ * dq_quantize_rows_int4 -- greedy (or min/max) row-wise INT4 quantization.
+ * ("Post-Training 4-bit Quantization on Embedding Tables", 提出的方法 / proposed
+ * method, bullets 1-2.)
+ *
+ *   x           [n_rows][x_ld] binary32, row-major; the first d of each row are used
+ *   n_rows      >= 0
+ *   d           1..DQ_MAX_D
+ *   x_ld        >= d, in elements
+ *   codes       [n_rows][codes_ld] bytes (output); only the first (d+1)/2 of a row are written
+ *   codes_ld    >= (d + 1) / 2, in bytes
+ *   scale_bias  [n_rows][2] binary16 bit patterns (output)
+ *   row_loss    [n_rows] binary32 (output, nullable): the search loss L at the chosen pair
+ *   best_ij     [n_rows][2] uint8 (output, nullable): the chosen grid indices (i*, j*)
+ *   mode        DQ_MODE_GREEDY or DQ_MODE_MINMAX
+ *   d_flags     device uint32 (nullable): DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW
+ *   cuda_stream cudaStream_t
+ *
+ * Rows with non-finite values or with a scale/bias beyond binary16's range give
+ * unspecified (but memory-safe) results.
+ */
+dq_status dq_quantize_rows_int4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld,
+                                uint8_t *codes, int64_t codes_ld, uint16_t *scale_bias,
+                                float *row_loss, uint8_t *best_ij, int32_t mode,
+                                uint32_t *d_flags, void *cuda_stream);
+
+/*
+ * dq_dequantize_rows -- out[r][k] = fma(q_k, scale, bias) in binary32.
+ * ("Post-Training 4-bit Quantization on Embedding Tables", 提出的方法 / proposed
+ * method, bullet 2: the FP16 scale and bias decode each row.)
+ *
+ *   codes, codes_ld, scale_bias   packed rows as above (inputs)
+ *   n_rows >= 0, d in 1..DQ_MAX_D
+ *   out         [n_rows][out_ld] binary32 (output), out_ld >= d elements
+ */
+dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint16_t *scale_bias,
+                             int64_t n_rows, int32_t d, float *out, int64_t out_ld,
+                             void *cuda_stream);
+
+/*
+ * dq_embbag_int4_fwd -- sum-pooled lookup over n_tables packed tables sharing d.
+ * ("Deep Learning Recommendation Model for Personalization and Recommendation
+ * Systems", 提出的方法 / proposed method, bullet 1.)
+ *
+ *   tables      HOST array of n_tables dq_table (1..DQ_MAX_TABLES); its contents are
+ *               copied at the call, the array may be reused on return
+ *   d           1..DQ_MAX_D
+ *   indices     int32 ids, table-relative
+ *   offsets     int32 [n_tables*batch + 1], table-major: bag (t, b) is
+ *               indices[offsets[t*batch + b] .. offsets[t*batch + b + 1]); indices
+ *               holds offsets[n_tables*batch] ids. A bag whose offsets decrease or
+ *               leave [0, offsets[n_tables*batch]] is clamped into that range (empty
+ *               if they decrease) and flagged DQ_FLAG_BAD_OFFSETS
+ *   batch       >= 0
+ *   out         [batch][n_tables*d] binary32 (output): out[b][t*d + k] is the binary32
+ *               sum over the bag of fma(q_k, scale, bias); an empty bag gives +0
+ *   d_flags     device uint32 (nullable): DQ_FLAG_BAD_INDEX, DQ_FLAG_BAD_OFFSETS
+ *
+ * The sum is accumulated in binary32 in id order. A bag of one id returns that
+ * row's dequantized values exactly.
+ */
+dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d,
+                             const int32_t *indices, const int32_t *offsets, int32_t batch,
+                             float *out, uint32_t *d_flags, void *cuda_stream);
+
+/* Static text for a status code. */
+const char *dq_status_string(dq_status s);
+
+/* The calling thread's last error message ("" if none); valid until its next call. */
+const char *dq_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int32_t dq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DQ_H */

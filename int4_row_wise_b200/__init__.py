@@ -1,0 +1,201 @@
+"""int4_row_wise_b200 -- row-wise INT4 quantization of embedding tables and the
+sum-pooled INT4 embedding bag, as CUDA kernels for B200 (sm_100a).
+
+This module is a thin binding over libdq.so's C ABI (include/dq.h): it marshals
+arguments (torch CUDA tensors -> device pointers, the current torch stream) and
+turns status codes into exceptions. Every step of the computation runs in
+libdq's kernels; there is no CPU path. If libdq.so is missing, the first call
+raises DqError (build it with `python -m int4_row_wise_b200.build`).
+
+Low-level calls with the C names:
+    dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd,
+    dq_status_string, dq_last_error, dq_version
+Convenience wrappers that allocate their outputs with torch:
+    quantize_rows, dequantize_rows, embbag
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import NamedTuple, Optional, Sequence
+
+__all__ = [
+    "DQ_OK", "DQ_ERR_INVALID_ARG", "DQ_ERR_UNSUPPORTED", "DQ_ERR_CUDA",
+    "DQ_MODE_GREEDY", "DQ_MODE_MINMAX",
+    "DQ_FLAG_BAD_INDEX", "DQ_FLAG_BAD_OFFSETS", "DQ_FLAG_NONFINITE", "DQ_FLAG_FP16_OVERFLOW",
+    "DQ_MAX_D", "DQ_MAX_TABLES", "DqError", "PackedTable", "lib_path", "load",
+    "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd",
+    "dq_status_string", "dq_last_error", "dq_version",
+    "quantize_rows", "dequantize_rows", "embbag",
+]
+
+DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA = 0, 1, 2, 3
+DQ_MODE_GREEDY, DQ_MODE_MINMAX = 0, 1
+DQ_FLAG_BAD_INDEX, DQ_FLAG_BAD_OFFSETS, DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW = 1, 2, 4, 8
+DQ_MAX_D, DQ_MAX_TABLES = 1024, 64
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libdq.so")
+_lock = threading.Lock()
+_lib = None
+
+
+class DqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(message)
+        self.status = status
+
+
+class _Table(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scale_bias", ctypes.c_void_p),
+                ("n_rows", ctypes.c_int64), ("codes_ld", ctypes.c_int64)]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def load():
+    """The loaded libdq (ctypes.CDLL); raises DqError if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise DqError(DQ_ERR_UNSUPPORTED,
+                              f"libdq.so not found at {_LIB_PATH}; build it with "
+                              "`python -m int4_row_wise_b200.build`")
+            L = ctypes.CDLL(_LIB_PATH)
+            vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+            L.dq_quantize_rows_int4.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, i32, vp, vp]
+            L.dq_quantize_rows_int4.restype = ctypes.c_int
+            L.dq_dequantize_rows.argtypes = [vp, i64, vp, i64, i32, vp, i64, vp]
+            L.dq_dequantize_rows.restype = ctypes.c_int
+            L.dq_embbag_int4_fwd.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp]
+            L.dq_embbag_int4_fwd.restype = ctypes.c_int
+            L.dq_status_string.argtypes, L.dq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+            L.dq_last_error.argtypes, L.dq_last_error.restype = [], ctypes.c_char_p
+            L.dq_version.argtypes, L.dq_version.restype = [], i32
+            _lib = L
+    return _lib
+
+
+def _ptr(a) -> Optional[int]:
+    """Device address of a CUDA tensor; ints pass through; None stays NULL."""
+    if a is None:
+        return None
+    if isinstance(a, int):
+        return a
+    if not a.is_cuda:
+        raise DqError(DQ_ERR_INVALID_ARG, "libdq takes CUDA tensors (device pointers)")
+    return a.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream if torch.cuda.is_available() else None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, what: str) -> None:
+    if status != DQ_OK:
+        L = load()
+        raise DqError(status, f"{what}: {L.dq_status_string(status).decode()}: {L.dq_last_error().decode()}")
+
+
+def dq_status_string(status: int) -> str:
+    return load().dq_status_string(status).decode()
+
+
+def dq_last_error() -> str:
+    return load().dq_last_error().decode()
+
+
+def dq_version() -> int:
+    return int(load().dq_version())
+
+
+def dq_quantize_rows_int4(x, n_rows: int, d: int, x_ld: int, codes, codes_ld: int, scale_bias,
+                          row_loss=None, best_ij=None, mode: int = DQ_MODE_GREEDY, d_flags=None,
+                          stream=None) -> None:
+    """C: dq_quantize_rows_int4. Tensors (or raw device addresses) for every buffer."""
+    st = load().dq_quantize_rows_int4(_ptr(x), n_rows, d, x_ld, _ptr(codes), codes_ld, _ptr(scale_bias),
+                                      _ptr(row_loss), _ptr(best_ij), mode, _ptr(d_flags), _stream(stream))
+    _check(st, "dq_quantize_rows_int4")
+
+
+def dq_dequantize_rows(codes, codes_ld: int, scale_bias, n_rows: int, d: int, out, out_ld: int,
+                       stream=None) -> None:
+    """C: dq_dequantize_rows."""
+    st = load().dq_dequantize_rows(_ptr(codes), codes_ld, _ptr(scale_bias), n_rows, d, _ptr(out), out_ld,
+                                   _stream(stream))
+    _check(st, "dq_dequantize_rows")
+
+
+class PackedTable(NamedTuple):
+    """A packed INT4 table on the device: codes uint8 [n, codes_ld], scale_bias int16 [n, 2]
+    (binary16 bit patterns)."""
+    codes: object
+    scale_bias: object
+
+    @property
+    def n_rows(self) -> int:
+        return int(self.codes.shape[0])
+
+
+def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, out, d_flags=None,
+                       stream=None) -> None:
+    """C: dq_embbag_int4_fwd. tables: PackedTable (or (codes, scale_bias)) per table."""
+    arr = (_Table * max(len(tables), 1))()
+    for t, tab in enumerate(tables):
+        codes, sb = tab[0], tab[1]
+        ld = int(codes.stride(0)) if codes.dim() == 2 else 0
+        arr[t] = _Table(_ptr(codes), _ptr(sb), int(codes.shape[0]), ld)
+    st = load().dq_embbag_int4_fwd(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
+                                   _ptr(offsets), batch, _ptr(out), _ptr(d_flags), _stream(stream))
+    _check(st, "dq_embbag_int4_fwd")
+
+
+# -------------------------------------------------------------------------
+# convenience wrappers (torch allocates the outputs on the input's device)
+# -------------------------------------------------------------------------
+
+def _codes_ld(d: int) -> int:
+    cb = (d + 1) // 2
+    return cb if cb < 16 else (cb + 15) // 16 * 16
+
+
+def quantize_rows(x, mode: int = DQ_MODE_GREEDY, with_loss: bool = True, d_flags=None, stream=None):
+    """x: CUDA float32 [n, d] (unit stride along d). Returns (codes uint8 [n, codes_ld],
+    scale_bias int16 [n, 2], row_loss float32 [n] or None, best_ij uint8 [n, 2] or None)."""
+    import torch
+    if x.dim() != 2 or x.dtype != torch.float32 or (x.shape[0] > 1 and x.stride(1) != 1):
+        raise DqError(DQ_ERR_INVALID_ARG, "x must be a float32 [n, d] tensor with unit stride along d")
+    n, d = x.shape
+    cld = _codes_ld(d)
+    codes = torch.empty((n, cld), dtype=torch.uint8, device=x.device)
+    sb = torch.empty((n, 2), dtype=torch.int16, device=x.device)
+    loss = torch.empty(n, dtype=torch.float32, device=x.device) if with_loss else None
+    ij = torch.empty((n, 2), dtype=torch.uint8, device=x.device) if with_loss else None
+    ld = x.stride(0) if n > 1 else d
+    dq_quantize_rows_int4(x, n, d, ld, codes, cld, sb, loss, ij, mode, d_flags, stream)
+    return codes, sb, loss, ij
+
+
+def dequantize_rows(codes, scale_bias, d: int, stream=None):
+    import torch
+    n = codes.shape[0]
+    out = torch.empty((n, d), dtype=torch.float32, device=codes.device)
+    dq_dequantize_rows(codes, codes.stride(0) if n > 1 else codes.shape[1], scale_bias, n, d, out, d, stream)
+    return out
+
+
+def embbag(tables: Sequence, d: int, indices, offsets, batch: int, d_flags=None, stream=None):
+    """Sum-pooled lookup; returns float32 [batch, len(tables) * d]."""
+    import torch
+    out = torch.empty((batch, len(tables) * d), dtype=torch.float32, device=indices.device)
+    dq_embbag_int4_fwd(tables, d, indices, offsets, batch, out, d_flags, stream)
+    return out

@@ -1,0 +1,200 @@
+// dq_api.cu -- the C ABI of libdq (declared in include/dq.h): host-side argument
+// validation, device checks and kernel dispatch. Every argument is checked before
+// anything is enqueued; the library allocates no memory.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <string>
+
+#include "dq_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+dq_status fail(dq_status s, const char *fmt, ...)
+{
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return s;
+}
+
+dq_status ok()
+{
+    g_last_error.clear();
+    return DQ_OK;
+}
+
+// Test hook: DQ_FAULT_INJECT=launch makes every entry point that would launch a
+// kernel return DQ_ERR_CUDA instead, with nothing enqueued.
+bool fault_injected()
+{
+    const char *v = getenv("DQ_FAULT_INJECT");
+    return v && strcmp(v, "launch") == 0;
+}
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];  // 0 = unknown, -1 = unsupported, else the SM count
+
+// Checks that the current device is an sm_100-class part; returns its SM count.
+dq_status current_device(int *num_sms)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return fail(DQ_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kMaxDevices)
+        return fail(DQ_ERR_UNSUPPORTED, "device ordinal %d beyond the library's table", dev);
+    int sms = g_sms[dev].load(std::memory_order_relaxed);
+    if (sms == 0) {
+        int major = 0, count = 0;
+        if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+            (e = cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return fail(DQ_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        sms = major == 10 ? count : -1;
+        g_sms[dev].store(sms, std::memory_order_relaxed);
+    }
+    if (sms < 0)
+        return fail(DQ_ERR_UNSUPPORTED, "device %d is not an sm_100 (B200-class) GPU", dev);
+    *num_sms = sms;
+    return DQ_OK;
+}
+
+dq_status launched(cudaError_t e, const char *what)
+{
+    if (e != cudaSuccess)
+        return fail(DQ_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+    return ok();
+}
+
+} // namespace
+
+extern "C" {
+
+dq_status dq_quantize_rows_int4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, uint8_t *codes,
+                                int64_t codes_ld, uint16_t *scale_bias, float *row_loss, uint8_t *best_ij,
+                                int32_t mode, uint32_t *d_flags, void *cuda_stream)
+{
+    if (n_rows < 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (x_ld < d)
+        return fail(DQ_ERR_INVALID_ARG, "x_ld = %lld < d = %d", (long long)x_ld, d);
+    if (codes_ld < (d + 1) / 2)
+        return fail(DQ_ERR_INVALID_ARG, "codes_ld = %lld < (d+1)/2 = %d", (long long)codes_ld, (d + 1) / 2);
+    if (mode != DQ_MODE_GREEDY && mode != DQ_MODE_MINMAX)
+        return fail(DQ_ERR_INVALID_ARG, "mode = %d is neither DQ_MODE_GREEDY nor DQ_MODE_MINMAX", mode);
+    if (n_rows > 0 && (!x || !codes || !scale_bias))
+        return fail(DQ_ERR_INVALID_ARG, "x, codes and scale_bias must be non-NULL when n_rows > 0");
+    if (n_rows > ((int64_t)1 << 40))
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld beyond 2^40", (long long)n_rows);
+    if (n_rows == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::QuantArgs a{x, n_rows, x_ld, d, codes, codes_ld, scale_bias, row_loss, best_ij, d_flags};
+    return launched(dq::launch_quantize(a, mode, sms, (cudaStream_t)cuda_stream), "quantize");
+}
+
+dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint16_t *scale_bias,
+                             int64_t n_rows, int32_t d, float *out, int64_t out_ld, void *cuda_stream)
+{
+    if (n_rows < 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (codes_ld < (d + 1) / 2)
+        return fail(DQ_ERR_INVALID_ARG, "codes_ld = %lld < (d+1)/2 = %d", (long long)codes_ld, (d + 1) / 2);
+    if (out_ld < d)
+        return fail(DQ_ERR_INVALID_ARG, "out_ld = %lld < d = %d", (long long)out_ld, d);
+    if (n_rows > 0 && (!codes || !scale_bias || !out))
+        return fail(DQ_ERR_INVALID_ARG, "codes, scale_bias and out must be non-NULL when n_rows > 0");
+    if (n_rows == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::DequantArgs a{codes, codes_ld, scale_bias, n_rows, d, out, out_ld};
+    return launched(dq::launch_dequantize(a, sms, (cudaStream_t)cuda_stream), "dequantize");
+}
+
+dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d, const int32_t *indices,
+                             const int32_t *offsets, int32_t batch, float *out, uint32_t *d_flags,
+                             void *cuda_stream)
+{
+    if (n_tables < 1 || n_tables > DQ_MAX_TABLES)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables = %d outside [1, %d]", n_tables, DQ_MAX_TABLES);
+    if (!tables)
+        return fail(DQ_ERR_INVALID_ARG, "tables must be non-NULL");
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (batch < 0)
+        return fail(DQ_ERR_INVALID_ARG, "batch = %d < 0", batch);
+    if ((int64_t)n_tables * batch + 1 > INT32_MAX)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables * batch + 1 offsets exceed int32 indexing");
+    dq::BagTables tabs;
+    memset(&tabs, 0, sizeof tabs);
+    for (int t = 0; t < n_tables; ++t) {
+        const dq_table &tb = tables[t];
+        if (tb.n_rows < 0)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].n_rows = %lld < 0", t, (long long)tb.n_rows);
+        if (tb.codes_ld < (d + 1) / 2)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].codes_ld = %lld < (d+1)/2 = %d", t,
+                        (long long)tb.codes_ld, (d + 1) / 2);
+        if (tb.n_rows > 0 && (!tb.codes || !tb.scale_bias))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codes and scale_bias must be non-NULL", t);
+        tabs.codes[t] = tb.codes;
+        tabs.scale_bias[t] = tb.scale_bias;
+        tabs.n_rows[t] = tb.n_rows;
+        tabs.codes_ld[t] = tb.codes_ld;
+    }
+    if (batch > 0 && (!indices || !offsets || !out))
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
+    if (batch == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::BagArgs a{n_tables, d, batch, indices, offsets, out, d_flags};
+    return launched(dq::launch_embbag(tabs, a, sms, (cudaStream_t)cuda_stream), "embbag");
+}
+
+const char *dq_status_string(dq_status s)
+{
+    switch (s) {
+    case DQ_OK: return "DQ_OK";
+    case DQ_ERR_INVALID_ARG: return "DQ_ERR_INVALID_ARG: invalid argument";
+    case DQ_ERR_UNSUPPORTED: return "DQ_ERR_UNSUPPORTED: unsupported device or request";
+    case DQ_ERR_CUDA: return "DQ_ERR_CUDA: CUDA error";
+    }
+    return "unknown dq_status";
+}
+
+const char *dq_last_error(void)
+{
+    return g_last_error.c_str();
+}
+
+int32_t dq_version(void)
+{
+    return 10000;
+}
+
+} // extern "C"

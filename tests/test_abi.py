@@ -1,0 +1,115 @@
+"""The C-ABI boundary without a GPU: libdq.so loads, exports every function
+include/dq.h declares, and rejects bad arguments on the host before touching
+the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import int4_row_wise_b200 as dq
+from int4_row_wise_b200 import build as dqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    dqbuild.build()
+    return dq.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "dq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(dq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert {"dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd",
+            "dq_status_string"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+    out = os.popen(f"nm -D --defined-only {dq.lib_path()}").read()
+    exported = set(re.findall(r"\bT (dq_[a-z0-9_]+)$", out, flags=re.M))
+    assert set(names) <= exported
+
+
+def test_status_strings_and_version(L):
+    assert dq.dq_status_string(dq.DQ_OK) == "DQ_OK"
+    assert "INVALID" in dq.dq_status_string(dq.DQ_ERR_INVALID_ARG)
+    assert "CUDA" in dq.dq_status_string(dq.DQ_ERR_CUDA)
+    assert dq.dq_version() == 10000
+
+
+NULL = None
+
+
+@pytest.mark.parametrize("args,msg", [
+    ((NULL, -1, 16, 16, NULL, 8, NULL, NULL, NULL, 0, NULL, NULL), "n_rows"),
+    ((NULL, 4, 0, 16, NULL, 8, NULL, NULL, NULL, 0, NULL, NULL), "d = 0"),
+    ((NULL, 4, 1025, 1025, NULL, 513, NULL, NULL, NULL, 0, NULL, NULL), "d = 1025"),
+    ((NULL, 4, 16, 15, NULL, 8, NULL, NULL, NULL, 0, NULL, NULL), "x_ld"),
+    ((NULL, 4, 16, 16, NULL, 7, NULL, NULL, NULL, 0, NULL, NULL), "codes_ld"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, NULL, 2, NULL, NULL), "mode"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, NULL, 0, NULL, NULL), "non-NULL"),
+])
+def test_quantize_rejects(L, args, msg):
+    assert L.dq_quantize_rows_int4(*args) == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
+def test_zero_rows_is_a_noop(L):
+    assert L.dq_quantize_rows_int4(NULL, 0, 16, 16, NULL, 8, NULL, NULL, NULL, 0, NULL, NULL) == dq.DQ_OK
+    assert L.dq_dequantize_rows(NULL, 8, NULL, 0, 16, NULL, 16, NULL) == dq.DQ_OK
+    t = (dq._Table * 1)(dq._Table(None, None, 0, 8))
+    assert L.dq_embbag_int4_fwd(ctypes.cast(t, ctypes.c_void_p), 1, 16, NULL, NULL, 0, NULL, NULL, NULL) == dq.DQ_OK
+
+
+@pytest.mark.parametrize("args,msg", [
+    ((NULL, 8, NULL, -1, 16, NULL, 16, NULL), "n_rows"),
+    ((NULL, 7, NULL, 3, 16, NULL, 16, NULL), "codes_ld"),
+    ((NULL, 8, NULL, 3, 16, NULL, 15, NULL), "out_ld"),
+    ((NULL, 8, NULL, 3, 2000, NULL, 2000, NULL), "d = 2000"),
+    ((NULL, 8, NULL, 3, 16, NULL, 16, NULL), "non-NULL"),
+])
+def test_dequantize_rejects(L, args, msg):
+    assert L.dq_dequantize_rows(*args) == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
+def _tables(*specs):
+    arr = (dq._Table * max(len(specs), 1))(*[dq._Table(*s) for s in specs])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+@pytest.mark.parametrize("tabspec,T,d,batch,msg", [
+    ([(None, None, 10, 8)], 0, 16, 4, "n_tables = 0"),
+    ([(None, None, 10, 8)], 65, 16, 4, "n_tables = 65"),
+    ([(None, None, 10, 8)], 1, 16, -1, "batch"),
+    ([(None, None, -1, 8)], 1, 16, 4, "n_rows"),
+    ([(None, None, 10, 7)], 1, 16, 4, "codes_ld"),
+    ([(None, None, 10, 8)], 1, 16, 4, "non-NULL"),
+    ([(1 << 20, 1 << 21, 10, 8)], 1, 16, 4, "indices"),
+    ([(1 << 20, 1 << 21, 10, 8)], 1, 0, 4, "d = 0"),
+])
+def test_embbag_rejects(L, tabspec, T, d, batch, msg):
+    p, keep = _tables(*tabspec)
+    assert L.dq_embbag_int4_fwd(p, T, d, None, None, batch, None, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
+def test_binding_raises_with_status(L):
+    with pytest.raises(dq.DqError) as ei:
+        dq.dq_quantize_rows_int4(None, 4, 0, 16, None, 8, None, stream=0)
+    assert ei.value.status == dq.DQ_ERR_INVALID_ARG and "d = 0" in str(ei.value)
+
+
+def test_library_sources_allocate_nothing():
+    # the library allocates no device or host memory of its own
+    import glob
+    for path in glob.glob(os.path.join(ROOT, "int4_row_wise_b200", "csrc", "*")):
+        src = open(path).read()
+        for call in ("cudaMalloc", "cudaFree", "cudaHostAlloc", "cudaMallocHost", "malloc(", "new "):
+            assert call not in src, (path, call)

@@ -1,0 +1,115 @@
+"""GPU parity of dq_dequantize_rows (bit-exact) and dq_embbag_int4_fwd (within
+1e-5 of the summed magnitudes, bit-exact for bags of one id) against the oracle.
+
+Lookup: "Deep Learning Recommendation Model for Personalization and
+Recommendation Systems", section 提出的方法 (proposed method), bullet 1."""
+import numpy as np
+import pytest
+import torch
+
+import int4_row_wise_b200 as dq
+import oracle
+from int4_row_wise_b200 import workloads as W
+from tests.gpu_util import bag_tolerance_check, gpu_quantize, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _packed(n, d, seed, codes_ld=None):
+    return W.random_packed_table(n, d, seed, codes_ld)
+
+
+@pytest.mark.parametrize("d,codes_ld,out_ld", [(16, 8, 16), (128, 64, 128), (256, 128, 256), (32, 16, 32),
+                                               (7, 4, 7), (16, 9, 16), (64, 32, 65), (1, 1, 1), (48, 24, 48)])
+def test_dequantize_bit_exact(cuda_device, d, codes_ld, out_ld):
+    n = 5003
+    codes, sb = _packed(n, d, d, codes_ld)
+    want = oracle.dequantize_rows(codes, sb, d)
+    out = torch.full((n, out_ld), -7.0, dtype=torch.float32, device="cuda")
+    dq.dq_dequantize_rows(to_dev(codes), codes_ld, to_dev(sb.view(np.int16)), n, d, out, out_ld)
+    got = out.cpu().numpy()
+    assert np.array_equal(got[:, :d].view(np.uint32), want.view(np.uint32))
+    assert np.all(got[:, d:] == -7.0)
+
+
+def _bags(T, B, rows, lo, hi, seed, bad=False):
+    r = np.random.default_rng(seed)
+    lens = r.integers(lo, hi + 1, T * B)
+    off = np.zeros(T * B + 1, np.int64)
+    off[1:] = np.cumsum(lens)
+    idx = np.concatenate([r.integers(0, rows[g // B], lens[g]) for g in range(T * B)]) if off[-1] else np.zeros(0)
+    idx = idx.astype(np.int32)
+    if bad and idx.size > 10:
+        idx[3] = -1
+        idx[7] = rows[0] + 5
+    return idx, off.astype(np.int32)
+
+
+def _gpu_bag(tabs, d, idx, off, B, flags=False):
+    dev_tabs = [dq.PackedTable(to_dev(c), to_dev(s.view(np.int16))) for c, s in tabs]
+    fl = torch.zeros(1, dtype=torch.int32, device="cuda") if flags else None
+    out = torch.full((B, len(tabs) * d), 123.0, dtype=torch.float32, device="cuda")
+    dq.dq_embbag_int4_fwd(dev_tabs, d, to_dev(idx if idx.size else np.zeros(1, np.int32)), to_dev(off), B,
+                          out, fl)
+    torch.cuda.synchronize()
+    return out.cpu().numpy(), (int(fl.item()) if flags else None)
+
+
+@pytest.mark.parametrize("d", [16, 32, 64, 128, 256, 512, 1024, 7, 48, 100])
+@pytest.mark.parametrize("pool", [(1, 1), (0, 3), (20, 80)])
+def test_bag_matches_oracle(cuda_device, d, pool):
+    T, B = 3, 97
+    rows = [500, 1000, 37]
+    tabs = [_packed(n, d, 10 * d + t, ((d + 1) // 2 + 15) // 16 * 16) for t, n in enumerate(rows)]
+    idx, off = _bags(T, B, rows, pool[0], pool[1], d)
+    got, _ = _gpu_bag(tabs, d, idx, off, B)
+    ref, mag, skipped = oracle.embbag(tabs, d, idx, off, B, with_abs_sum=True)
+    assert skipped == 0
+    bag_tolerance_check(got, ref, mag)
+    if pool == (1, 1):
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_bag_bad_ids_and_offsets(cuda_device):
+    d, T, B = 64, 2, 50
+    rows = [100, 100]
+    tabs = [_packed(n, d, 5 + t) for t, n in enumerate(rows)]
+    idx, off = _bags(T, B, rows, 1, 6, 3, bad=True)
+    off2 = off.copy()
+    off2[20] = off2[21] + 2   # bag 19 gets decreasing offsets... and bag 20 a longer span
+    got, fl = _gpu_bag(tabs, d, idx, off2, B, flags=True)
+    ref, mag, skipped = oracle.embbag(tabs, d, idx, off2, B, with_abs_sum=True)
+    assert skipped > 0
+    assert fl & dq.DQ_FLAG_BAD_INDEX and fl & dq.DQ_FLAG_BAD_OFFSETS
+    bag_tolerance_check(got, ref, mag)
+    got, fl = _gpu_bag(tabs, d, *_bags(T, B, rows, 1, 6, 4), B, flags=True)
+    assert fl == 0
+
+
+def test_tiny_workload_end_to_end(cuda_device):
+    """Quantize the tiny table on the GPU, then look it up on the GPU; the oracle
+    sums the same packed table."""
+    wl = W.workload("tiny")
+    x = W.table_rows(wl, 0)
+    codes, sb, _, _, _ = gpu_quantize(x)
+    idx, off = W.lookup_batch(wl)
+    got, _ = _gpu_bag([(codes, sb)], wl.d, idx, off, wl.batch)
+    ref, mag, _ = oracle.embbag([(codes, sb)], wl.d, idx, off, wl.batch, with_abs_sum=True)
+    bag_tolerance_check(got, ref, mag)
+    deq = torch.empty((x.shape[0], wl.d), dtype=torch.float32, device="cuda")
+    dq.dq_dequantize_rows(to_dev(codes), codes.shape[1], to_dev(sb.view(np.int16)), x.shape[0], wl.d, deq, wl.d)
+    assert np.array_equal(deq.cpu().numpy().view(np.uint32), oracle.dequantize_rows(codes, sb, wl.d).view(np.uint32))
+
+
+@pytest.mark.parametrize("name", ["kaggle", "sweep-64"])
+def test_workload_batches_on_random_tables(cuda_device, name):
+    """A full lookup call of the workload (its ids, offsets and batch), over random
+    packed tables of its table sizes."""
+    wl = W.workload(name)
+    tabs = [_packed(n, wl.d, 1000 + t, ((wl.d + 1) // 2 + 15) // 16 * 16) for t, n in enumerate(wl.rows)]
+    idx, off = W.lookup_batch(wl)
+    got, _ = _gpu_bag(tabs, wl.d, idx, off, wl.batch)
+    ref, mag, _ = oracle.embbag(tabs, wl.d, idx, off, wl.batch, with_abs_sum=True)
+    bag_tolerance_check(got, ref, mag)
+    if wl.pooling == (1, 1):
+        assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
