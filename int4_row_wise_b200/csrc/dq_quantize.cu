@@ -9,19 +9,27 @@
 //
 // Layout: a row of d <= P = next_pow2(d) elements is held in registers by W lanes
 // of one warp, M = P / W contiguous elements per lane (M = 16 for P >= 16). The
-// search is pure FP32 ALU work: 337 loss evaluations x d elements per row, each
-// element ~10 instructions, two candidates evaluated side by side for ILP. The
-// loss is a pairwise sum: an in-lane binary tree over M elements, then an XOR
-// butterfly over the W lanes, which is the same recursive-halving order, so
-// every lane of the row gets the identical binary32 value.
+// search is pure FP32 ALU work: 337 loss evaluations x d elements per row. The two
+// candidates of a move are evaluated side by side (ILP), and the per-element work
+// runs on packed f32x2 FMA/ADD/MUL, which issue once for two lanes' worth of FP32
+// work: a lane pairs element m with element m + M/2, so the packed adds of the
+// error tree are exactly the pairwise (recursive-halving) order, and an XOR
+// butterfly over the W lanes finishes it. Every lane of a row gets the identical
+// binary32 loss.
 //
-// The code of an element during the search, q = clamp(rint((x - lo) / s), 0, 15)
-// with an IEEE quotient, is computed without a division: u = sat((x - lo) * rcp(w))
-// (w = hi - lo ~ 15 s), then rint(15 u) by a magic-number add. 15 u is within
-// 4e-6 of the exact quotient, so it rounds the same way as the IEEE quotient
-// unless it lies within 2^-16 of a half-integer; those rare elements are flagged
-// and recomputed with the IEEE division. The codes the search sees are therefore
-// exactly the IEEE ones.
+// Codes during the search: q = clamp(rint((x - lo) / s), 0, 15) needs an IEEE
+// quotient. The kernel instead forms u = sat(fma(x, r, -lo*r)) with r = rcp(w),
+// w = hi - lo (= 15 s up to one rounding), and rounds 15u with a magic-number add.
+// |15u - (x - lo)/s| <= 5.6e-6 + 9e-7 * |lo * r| (rcp error <= 1 ulp), so 15u rounds
+// like the IEEE quotient unless it lies within the margin 2^-16 + 2^-19 * |lo * r|
+// of a half-integer; such elements (a few in 10^5) are recomputed with IEEE
+// division. The codes the search sees are therefore exactly the IEEE ones.
+//
+// s = w / 15 uses Markstein's correction step for a known divisor (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Dev. 34(1), 1990): q0 = w * RN(1/15), rem = fma(-q0, 15, w),
+// s = fma(rem, RN(1/15), q0). It equals the IEEE quotient for every positive
+// normal binary32 w (checked exhaustively); the fast path only uses w >= 1e-36.
 #include <cfloat>
 
 #include "dq_internal.cuh"
@@ -33,9 +41,12 @@ constexpr float kSteps = 200.0f;         // grid steps over the row's range
 constexpr int kMoves = 168;              // moves while width > 0.16 * range
 constexpr float kLevels = 15.0f;         // 2^4 - 1
 constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23: x + kMagic rounds x in [0, 2^22) to an integer
-constexpr float kHardGap = 0.5f - 1.52587890625e-05f;  // flag |15u - q| beyond 0.5 - 2^-16
+constexpr float kInv15 = 1.0f / 15.0f;   // RN(1/15)
+constexpr float kGap0 = 0.5f - 1.52587890625e-05f;  // 0.5 - 2^-16
+constexpr float kGapLo = 1.9073486328125e-06f;     // 2^-19 per unit of |lo * r|
 constexpr float kFastWMin = 1.0e-36f;    // w in [kFastWMin, kFastWMax]: s normal, 1/w normal
 constexpr float kFastWMax = 1.0e36f;
+constexpr float kFastLoR = 65536.0f;     // |lo * r| above this: IEEE path
 
 __device__ __forceinline__ float rcp_approx(float x)
 {
@@ -44,11 +55,19 @@ __device__ __forceinline__ float rcp_approx(float x)
     return r;
 }
 
-__device__ __forceinline__ float mul_sat(float a, float b)
+__device__ __forceinline__ float fma_sat(float a, float b, float c)
 {
     float r;
-    asm("mul.rn.sat.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
     return r;
+}
+
+// w / 15 rounded to nearest even, for positive normal w (Markstein correction).
+__device__ __forceinline__ float div15(float w)
+{
+    const float q0 = __fmul_rn(w, kInv15);
+    const float rem = __fmaf_rn(-q0, kLevels, w);
+    return __fmaf_rn(rem, kInv15, q0);
 }
 
 // q = clamp(rint(fl(fl(x - lo) / s)), 0, 15) with an IEEE quotient; 0 when s == 0.
@@ -58,18 +77,6 @@ __device__ __forceinline__ float exact_code(float x, float lo, float s)
         return 0.0f;
     float q = rintf(__fdiv_rn(__fsub_rn(x, lo), s));
     return fminf(fmaxf(q, 0.0f), kLevels);
-}
-
-template <int M>
-__device__ __forceinline__ float tree_sum(float (&c)[M])
-{
-#pragma unroll
-    for (int w = 1; w < M; w <<= 1) {
-#pragma unroll
-        for (int k = 0; k < M; k += 2 * w)
-            c[k] = __fadd_rn(c[k], c[k + w]);
-    }
-    return c[0];
 }
 
 template <int W>
@@ -91,64 +98,155 @@ __device__ __forceinline__ void row_minmax(float &mn, float &mx)
     }
 }
 
-// Squared reconstruction errors of this lane's M elements for one clip range,
-// with IEEE codes (exact path).
-template <int M, bool FULL>
-__device__ __forceinline__ void errors_exact(const float (&v)[M], int kbase, int d, float lo, float s,
-                                             float (&c)[M])
+// One clip range [lo, hi] of the search, with what its elements share.
+struct Clip {
+    float lo, s;      // bias and scale of the candidate quantizer
+    float r, nlr;     // rcp(hi - lo) and -RN(lo * r): u = sat(fma(x, r, nlr))
+    float thr;        // |15u - q| above thr: too close to a rounding tie, recompute
+};
+
+__device__ __forceinline__ Clip clip_fast(float lo, float hi, float thr)
 {
+    Clip c;
+    c.lo = lo;
+    const float w = __fsub_rn(hi, lo);
+    c.r = rcp_approx(w);
+    c.nlr = __fmul_rn(-lo, c.r);
+    c.s = div15(w);
+    c.thr = thr;
+    return c;
+}
+
+__device__ __forceinline__ float sq_err_exact(float x, float lo, float s)
+{
+    const float q = exact_code(x, lo, s);
+    const float e = __fsub_rn(x, __fmaf_rn(q, s, lo));
+    return __fmul_rn(e, e);
+}
+
+// Element k of the lane sits in slot .x of pair k (k < H) or slot .y of pair k - H.
+template <int H, bool HAS_Y, bool FULL>
+__device__ __forceinline__ bool valid_x(int kbase, int h, int d) { return FULL || kbase + h < d; }
+template <int H, bool HAS_Y, bool FULL>
+__device__ __forceinline__ bool valid_y(int kbase, int h, int d) { return HAS_Y && (FULL || kbase + h + H < d); }
+
+// Squared errors of the lane's elements for one clip (packed f32x2). Sets `hard` if
+// an element's code must be recomputed with IEEE division.
+template <int H, bool HAS_Y, bool FULL>
+__device__ __forceinline__ void errors_packed(const float2 (&xp)[H], const Clip &c, int kbase, int d,
+                                              float2 (&C)[H], bool &hard)
+{
+    const float2 k15 = make_float2(kLevels, kLevels), kmag = make_float2(kMagic, kMagic);
+    const float2 km1 = make_float2(-1.0f, -1.0f);
+    const float2 ns2 = make_float2(-c.s, -c.s), lo2 = make_float2(c.lo, c.lo);
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        float q = exact_code(v[m], lo, s);
-        float xh = __fmaf_rn(q, s, lo);
-        float e = __fsub_rn(v[m], xh);
-        c[m] = (FULL || kbase + m < d) ? __fmul_rn(e, e) : 0.0f;
+    for (int h = 0; h < H; ++h) {
+        const float2 U = make_float2(fma_sat(xp[h].x, c.r, c.nlr), fma_sat(xp[h].y, c.r, c.nlr));
+        const float2 Z = __ffma2_rn(U, k15, kmag);     // kMagic + rint(15u)
+        const float2 NQ = __ffma2_rn(Z, km1, kmag);    // -q, exact
+        const float2 DD = __ffma2_rn(U, k15, NQ);      // 15u - q
+        hard |= fabsf(DD.x) > c.thr;
+        if (HAS_Y)
+            hard |= fabsf(DD.y) > c.thr;
+        const float2 XH = __ffma2_rn(NQ, ns2, lo2);    // q*s + lo, rounded once
+        const float2 E = __ffma2_rn(XH, km1, xp[h]);   // x - xhat
+        C[h] = __fmul2_rn(E, E);
+        if (!valid_x<H, HAS_Y, FULL>(kbase, h, d))
+            C[h].x = 0.0f;
+        if (!valid_y<H, HAS_Y, FULL>(kbase, h, d))
+            C[h].y = 0.0f;
     }
 }
 
-// The two candidate losses of one move, (lo_a, hi_a) and (lo_b, hi_b), for this
-// lane's elements (before the cross-lane butterfly).
-template <int M, bool FULL>
-__device__ __forceinline__ void lane_loss_pair(const float (&v)[M], int kbase, int d, float lo_a,
-                                               float hi_a, float lo_b, float hi_b, float &la, float &lb)
+// The tie distance 15u - q of one element, by the same operations as errors_packed.
+__device__ __forceinline__ float tie_distance(float x, const Clip &c)
 {
-    const float wa = __fsub_rn(hi_a, lo_a), wb = __fsub_rn(hi_b, lo_b);
-    const float sa = __fdiv_rn(wa, kLevels), sb = __fdiv_rn(wb, kLevels);
-    float ca[M], cb[M];
-    const bool fast = wa >= kFastWMin && wa <= kFastWMax && wb >= kFastWMin && wb <= kFastWMax;
-    bool hard_a = !fast, hard_b = !fast;
-    if (fast) {
-        const float ra = rcp_approx(wa), rb = rcp_approx(wb);
-        const float nsa = -sa, nsb = -sb;
+    const float u = fma_sat(x, c.r, c.nlr);
+    const float nq = __fmaf_rn(__fmaf_rn(u, kLevels, kMagic), -1.0f, kMagic);
+    return __fmaf_rn(u, kLevels, nq);
+}
+
+// Recomputes with IEEE division every element whose fast code was too close to a tie.
+template <int H, bool HAS_Y, bool FULL>
+__device__ __forceinline__ void errors_fixup(const float2 (&xp)[H], const Clip &c, int kbase, int d,
+                                             float2 (&C)[H])
+{
 #pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const float ta = __fsub_rn(v[m], lo_a), tb = __fsub_rn(v[m], lo_b);
-            const float ua = mul_sat(ta, ra), ub = mul_sat(tb, rb);
-            const float za = __fmaf_rn(ua, kLevels, kMagic), zb = __fmaf_rn(ub, kLevels, kMagic);
-            const float nqa = __fsub_rn(kMagic, za), nqb = __fsub_rn(kMagic, zb);   // -q, exact
-            const float da = __fmaf_rn(ua, kLevels, nqa), db = __fmaf_rn(ub, kLevels, nqb);
-            hard_a |= fabsf(da) > kHardGap;
-            hard_b |= fabsf(db) > kHardGap;
-            const float xa = __fmaf_rn(nqa, nsa, lo_a), xb = __fmaf_rn(nqb, nsb, lo_b);  // q*s + lo, once rounded
-            const float ea = __fsub_rn(v[m], xa), eb = __fsub_rn(v[m], xb);
-            ca[m] = (FULL || kbase + m < d) ? __fmul_rn(ea, ea) : 0.0f;
-            cb[m] = (FULL || kbase + m < d) ? __fmul_rn(eb, eb) : 0.0f;
+    for (int h = 0; h < H; ++h) {
+        if (valid_x<H, HAS_Y, FULL>(kbase, h, d) && fabsf(tie_distance(xp[h].x, c)) > c.thr)
+            C[h].x = sq_err_exact(xp[h].x, c.lo, c.s);
+        if (valid_y<H, HAS_Y, FULL>(kbase, h, d) && fabsf(tie_distance(xp[h].y, c)) > c.thr)
+            C[h].y = sq_err_exact(xp[h].y, c.lo, c.s);
+    }
+}
+
+// Every element with IEEE division (rows outside the fast path's range).
+template <int H, bool HAS_Y, bool FULL>
+__device__ __forceinline__ void errors_exact(const float2 (&xp)[H], float lo, float hi, int kbase, int d,
+                                             float2 (&C)[H])
+{
+    const float s = __fdiv_rn(__fsub_rn(hi, lo), kLevels);
+#pragma unroll
+    for (int h = 0; h < H; ++h) {
+        C[h].x = valid_x<H, HAS_Y, FULL>(kbase, h, d) ? sq_err_exact(xp[h].x, lo, s) : 0.0f;
+        C[h].y = valid_y<H, HAS_Y, FULL>(kbase, h, d) ? sq_err_exact(xp[h].y, lo, s) : 0.0f;
+    }
+}
+
+// Pairwise sum of the lane's squared errors: slot .x holds the first half of the
+// lane's elements, slot .y the second, so packed adds run both halves' trees.
+template <int H>
+__device__ __forceinline__ float tree_sum2(float2 (&C)[H])
+{
+#pragma unroll
+    for (int w = 1; w < H; w <<= 1) {
+#pragma unroll
+        for (int k = 0; k < H; k += 2 * w)
+            C[k] = __fadd2_rn(C[k], C[k + w]);
+    }
+    return __fadd_rn(C[0].x, C[0].y);
+}
+
+// The 168 moves of the greedy walk. FAST: division-free codes with tie fix-up;
+// otherwise IEEE division for every element. All lanes of a row see the same losses.
+template <int H, bool HAS_Y, bool FULL, bool FAST, int W>
+__device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, int d, float mn, float mx,
+                                            float step, float thr, float &lbest, float &fbi, float &fbj)
+{
+    float fi = 0.0f, fj = 0.0f;  // grid indices as exact small floats (i + j <= 168)
+    float lo_i = __fmaf_rn(0.0f, step, mn), hi_j = __fmaf_rn(-0.0f, step, mx);
+    float lo_i1 = __fmaf_rn(1.0f, step, mn), hi_j1 = __fmaf_rn(-1.0f, step, mx);
+    for (int mv = 0; mv < kMoves; ++mv) {
+        // left candidate (i+1, j) = a, right candidate (i, j+1) = b
+        float2 Ca[H], Cb[H];
+        if constexpr (FAST) {
+            const Clip ca = clip_fast(lo_i1, hi_j, thr), cb = clip_fast(lo_i, hi_j1, thr);
+            bool hard = false;
+            errors_packed<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca, hard);
+            errors_packed<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb, hard);
+            if (hard) {
+                errors_fixup<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca);
+                errors_fixup<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb);
+            }
+        } else {
+            errors_exact<H, HAS_Y, FULL>(xp, lo_i1, hi_j, kbase, d, Ca);
+            errors_exact<H, HAS_Y, FULL>(xp, lo_i, hi_j1, kbase, d, Cb);
         }
+        const float la = row_sum<W>(tree_sum2<H>(Ca));
+        const float lb = row_sum<W>(tree_sum2<H>(Cb));
+        const bool right = lb < la;  // ties move left
+        const float l = right ? lb : la;
+        fi = right ? fi : fi + 1.0f;
+        fj = right ? fj + 1.0f : fj;
+        lo_i = right ? lo_i : lo_i1;
+        hi_j = right ? hi_j1 : hi_j;
+        lo_i1 = __fmaf_rn(fi + 1.0f, step, mn);
+        hi_j1 = __fmaf_rn(-(fj + 1.0f), step, mx);
+        const bool better = l < lbest;  // the first lowest loss is kept
+        lbest = better ? l : lbest;
+        fbi = better ? fi : fbi;
+        fbj = better ? fj : fbj;
     }
-    if (hard_a)
-        errors_exact<M, FULL>(v, kbase, d, lo_a, sa, ca);
-    if (hard_b)
-        errors_exact<M, FULL>(v, kbase, d, lo_b, sb, cb);
-    la = tree_sum<M>(ca);
-    lb = tree_sum<M>(cb);
-}
-
-template <int M, bool FULL>
-__device__ __forceinline__ float lane_loss_one(const float (&v)[M], int kbase, int d, float lo, float hi)
-{
-    float c[M];
-    errors_exact<M, FULL>(v, kbase, d, lo, __fdiv_rn(__fsub_rn(hi, lo), kLevels), c);
-    return tree_sum<M>(c);
 }
 
 // One row per W lanes; M elements per lane; FULL: d == M * W (no padding);
@@ -156,6 +254,8 @@ __device__ __forceinline__ float lane_loss_one(const float (&v)[M], int kbase, i
 template <int M, int W, bool FULL, bool VEC>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, const int greedy)
 {
+    constexpr bool HAS_Y = M > 1;
+    constexpr int H = HAS_Y ? M / 2 : 1;
     const int sub = threadIdx.x & (W - 1);
     int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
     const bool active = row < a.n;
@@ -165,8 +265,10 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, c
     const int kbase = sub * M;
     const float *xr = a.x + row * a.ld + kbase;
 
-    float v[M];
+    // the lane's M elements: element k in xp[k].x (k < H) or xp[k - H].y
+    float2 xp[H];
     if constexpr (VEC) {
+        float v[M];
 #pragma unroll
         for (int m = 0; m < M; m += 4) {
             const float4 q4 = __ldg(reinterpret_cast<const float4 *>(xr + m));
@@ -175,55 +277,63 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, c
             v[m + 2] = q4.z;
             v[m + 3] = q4.w;
         }
+#pragma unroll
+        for (int h = 0; h < H; ++h)
+            xp[h] = make_float2(v[h], v[h + H]);
     } else {
 #pragma unroll
-        for (int m = 0; m < M; ++m)
-            v[m] = (FULL || kbase + m < d) ? __ldg(xr + m) : 0.0f;
+        for (int h = 0; h < H; ++h) {
+            xp[h].x = valid_x<H, HAS_Y, FULL>(kbase, h, d) ? __ldg(xr + h) : 0.0f;
+            xp[h].y = valid_y<H, HAS_Y, FULL>(kbase, h, d) ? __ldg(xr + h + H) : 0.0f;
+        }
     }
 
     float mn = FLT_MAX, mx = -FLT_MAX;
     bool nonfinite = false;
 #pragma unroll
-    for (int m = 0; m < M; ++m) {
-        if (FULL || kbase + m < d) {
-            mn = fminf(mn, v[m]);
-            mx = fmaxf(mx, v[m]);
-            nonfinite |= !isfinite(v[m]);
+    for (int h = 0; h < H; ++h) {
+        if (valid_x<H, HAS_Y, FULL>(kbase, h, d)) {
+            mn = fminf(mn, xp[h].x);
+            mx = fmaxf(mx, xp[h].x);
+            nonfinite |= !isfinite(xp[h].x);
+        }
+        if (valid_y<H, HAS_Y, FULL>(kbase, h, d)) {
+            mn = fminf(mn, xp[h].y);
+            mx = fmaxf(mx, xp[h].y);
+            nonfinite |= !isfinite(xp[h].y);
         }
     }
     row_minmax<W>(mn, mx);
 
     const float range = __fsub_rn(mx, mn);
     const float step = __fdiv_rn(range, kSteps);
-    float lbest = row_sum<W>(lane_loss_one<M, FULL>(v, kbase, d, mn, mx));
-    int i = 0, j = 0, bi = 0, bj = 0;
-    if (greedy) {
-        for (int mv = 0; mv < kMoves; ++mv) {
-            const float lo_l = __fmaf_rn((float)(i + 1), step, mn), hi_l = __fmaf_rn(-(float)j, step, mx);
-            const float lo_r = __fmaf_rn((float)i, step, mn), hi_r = __fmaf_rn(-(float)(j + 1), step, mx);
-            float ll, lr;
-            lane_loss_pair<M, FULL>(v, kbase, d, lo_l, hi_l, lo_r, hi_r, ll, lr);
-            ll = row_sum<W>(ll);
-            lr = row_sum<W>(lr);
-            float l;
-            if (lr < ll) {
-                ++j;
-                l = lr;
-            } else {
-                ++i;
-                l = ll;
-            }
-            if (l < lbest) {
-                lbest = l;
-                bi = i;
-                bj = j;
-            }
-        }
+    float lbest;
+    {
+        float2 C0[H];
+        errors_exact<H, HAS_Y, FULL>(xp, mn, mx, kbase, d, C0);
+        lbest = row_sum<W>(tree_sum2<H>(C0));
     }
+    float fbi = 0.0f, fbj = 0.0f;
+    // A constant row has loss 0 at every grid point: the walk cannot change (0, 0).
+    if (greedy && range != 0.0f) {
+        // Fast path, decided once per row. Every candidate has |lo| <= max(|xmin|, |xmax|)
+        // and width > 30 * step (the walk stops at 32 steps; when K <= 2^16 the grid
+        // points' rounding costs less than 0.25 step), so K bounds |lo * rcp(hi - lo)|
+        // for the whole walk and sets the tie margin.
+        const float w_min = __fmul_rn(step, 30.0f);
+        const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
+        const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
+        const float thr = __fmaf_rn(K, -kGapLo, kGap0);
+        if (fast)
+            greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, thr, lbest, fbi, fbj);
+        else
+            greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, thr, lbest, fbi, fbj);
+    }
+    const int bi = (int)fbi, bj = (int)fbj;
 
     // Final parameters in binary16 and the codes with IEEE division.
-    const float lo = __fmaf_rn((float)bi, step, mn);
-    const float hi = __fmaf_rn(-(float)bj, step, mx);
+    const float lo = __fmaf_rn(fbi, step, mn);
+    const float hi = __fmaf_rn(-fbj, step, mx);
     const float s = __fdiv_rn(__fsub_rn(hi, lo), kLevels);
     const __half s16 = __float2half_rn(s), b16 = __float2half_rn(lo);
     const float S = __half2float(s16), B = __half2float(b16);
@@ -231,10 +341,13 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, c
 #pragma unroll
     for (int m = 0; m < (M + 1) / 2; ++m) {
         const int k0 = 2 * m, k1 = 2 * m + 1;
-        const unsigned q0 = (FULL || kbase + k0 < d) ? (unsigned)exact_code(v[k0], B, S) : 0u;
+        const float x0 = k0 < H ? xp[k0 % H].x : xp[(k0 - H) % H].y;
+        const unsigned q0 = (FULL || kbase + k0 < d) ? (unsigned)exact_code(x0, B, S) : 0u;
         unsigned q1 = 0u;
-        if (k1 < M && (FULL || kbase + k1 < d))
-            q1 = (unsigned)exact_code(v[k1], B, S);
+        if (k1 < M && (FULL || kbase + k1 < d)) {
+            const float x1 = k1 < H ? xp[k1 % H].x : xp[(k1 - H) % H].y;
+            q1 = (unsigned)exact_code(x1, B, S);
+        }
         packed[m] = (uint8_t)(q0 | (q1 << 4));
     }
     if (!active)
