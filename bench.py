@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 from int4_row_wise_b200 import workloads as W  # noqa: E402
 
+LARGE_BYTES = 8 << 30  # fp32 tables above this are generated in parallel and skip the e2e leg
 METRIC = "quantized rows/s and INT4 embedding-bag GB/s (fraction of B200 HBM roofline)"
 FLOPS_PER_ELEMENT_EVAL = 10      # sub, div, rint, 2 clamps, mul, add, sub, mul, add
 EVALS_PER_ROW = 1 + 2 * 168      # initial clip + two candidates per move
@@ -162,8 +163,15 @@ class OracleBench:
         n_sample = int(max(self.cores * 16, min(wl.total_rows, target_s * self.cores / self.per_row_core * 0.8)))
         share = np.array(wl.rows, dtype=np.float64) / wl.total_rows
         per_table = np.minimum(np.maximum(1, np.round(share * n_sample).astype(np.int64)), np.array(wl.rows))
-        x = np.concatenate([W.sample_rows(wl, t, np.sort(rng.choice(wl.rows[t], int(k), replace=False)))
-                            for t, k in enumerate(per_table)])
+        xs = []
+        for t, k in enumerate(per_table):
+            # rows drawn from at most 4 random blocks of the table (cheap to regenerate)
+            nb = W.n_blocks(wl, t)
+            blocks = rng.choice(nb, min(nb, 4), replace=False)
+            cand = np.concatenate([np.arange(b * W.BLOCK_ROWS, min((b + 1) * W.BLOCK_ROWS, wl.rows[t]))
+                                   for b in blocks])
+            xs.append(W.sample_rows(wl, t, np.sort(rng.choice(cand, min(int(k), cand.size), replace=False))))
+        x = np.concatenate(xs)
         t0 = time.perf_counter()
         codes, sb, _, _ = oracle.quantize_rows(x, nthreads=self.cores)
         tq = time.perf_counter() - t0
@@ -175,7 +183,8 @@ class OracleBench:
         tbag = time.perf_counter() - t0
         n = x.shape[0]
         step_s = (tq + tdq) * wl.total_rows / n + tbag
-        sample = (f"{n} rows sampled across all {wl.n_tables} tables in proportion to their sizes "
+        sample = (f"{n} rows sampled across all {wl.n_tables} tables in proportion to their sizes (from <= 4 blocks "
+                  f"of {W.BLOCK_ROWS} rows per table) "
                   f"(quantize {tq:.2f} s + dequantize {tdq:.3f} s, scaled to {wl.total_rows} rows) "
                   f"+ one full lookup call ({tbag:.3f} s)")
         return wl.total_rows / step_s, step_s, sample
@@ -205,6 +214,25 @@ def run_reference(args, wl: W.Workload) -> None:
 
 
 # ---------------------------------------------------------------------------
+# multi-rank host logic (weak scaling, no collective on the data path)
+# ---------------------------------------------------------------------------
+def rank_workload(name: str, rank: int) -> W.Workload:
+    """Rank r quantizes its own independent set of tables: the workload drawn with seed r."""
+    return W.workload(name, seed=rank)
+
+
+def max_over_ranks(value: float, device) -> float:
+    """The max of a per-rank device time over all ranks (a no-op without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
 # the CUDA path
 # ---------------------------------------------------------------------------
 def run_gpu(args, wl: W.Workload) -> None:
@@ -226,9 +254,17 @@ def run_gpu(args, wl: W.Workload) -> None:
     dq.load()
 
     # --- inputs, generated on the host (seeded per rank) and made resident in HBM
-    wlr = W.workload(wl.name, seed=rank)
-    host_tables = [W.table_rows(wlr, t) for t in range(wlr.n_tables)]
-    xs = [torch.from_numpy(h).to(dev) for h in host_tables]
+    wlr = rank_workload(wl.name, rank)
+    big = wlr.total_rows * wlr.d * 4 > LARGE_BYTES
+    host_tables, xs = [], []
+    for t in range(wlr.n_tables):
+        if big:  # generated block-parallel into shared memory, uploaded, released
+            st = W.SharedTable(wlr, t)
+            xs.append(torch.from_numpy(st.array).to(dev))
+            st.close()
+        else:
+            host_tables.append(W.table_rows(wlr, t))
+            xs.append(torch.from_numpy(host_tables[-1]).to(dev))
     d = wlr.d
     cld = dq._codes_ld(d)
     codes = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wlr.rows]
@@ -244,13 +280,32 @@ def run_gpu(args, wl: W.Workload) -> None:
     launches_per_step = sum(1 for n in wlr.rows if n > 0) * 2 + 1
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Tables are spread over side streams (largest first, each to the least loaded
+    # stream) so the partly idle last wave of one table overlaps the next table.
+    side = [torch.cuda.Stream(dev) for _ in range(max(1, args.streams))]
+    load = [0] * len(side)
+    owner = [0] * wlr.n_tables
+    for t in sorted(range(wlr.n_tables), key=lambda t: -wlr.rows[t]):
+        k = min(range(len(side)), key=lambda i: load[i])
+        owner[t] = k
+        load[k] += wlr.rows[t]
+    fork = torch.cuda.Event()
+    joins = [torch.cuda.Event() for _ in side]
 
     def step(k: int, timed: bool):
         e = ev[k] if timed else None
         if e:
             e[0].record(stream)
-        for x, c, s in zip(xs, codes, sbs):
-            dq.dq_quantize_rows_int4(x, x.shape[0], d, d, c, cld, s, None, None, dq.DQ_MODE_GREEDY, None, stream)
+        fork.record(stream)
+        for sst in side:
+            sst.wait_event(fork)
+        for t in range(wlr.n_tables):
+            sst = side[owner[t]]
+            dq.dq_quantize_rows_int4(xs[t], xs[t].shape[0], d, d, codes[t], cld, sbs[t], None, None,
+                                     dq.DQ_MODE_GREEDY, None, sst)
+        for sst, j in zip(side, joins):
+            j.record(sst)
+            stream.wait_event(j)
         if e:
             e[1].record(stream)
         bi, bo = batches[k % n_batches]
@@ -286,10 +341,7 @@ def run_gpu(args, wl: W.Workload) -> None:
     dq_ms = sum(e[2].elapsed_time(e[3]) for e in ev)
     clocks = sampler.summary()
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     rows_all = wlr.total_rows * world * args.steps
     value = rows_all / (total_ms / 1e3)
@@ -309,7 +361,10 @@ def run_gpu(args, wl: W.Workload) -> None:
     hbm = _measured_hbm()
 
     # --- end to end through the public API with pinned host buffers
-    e2e = run_e2e(args, wlr, host_tables, batches_h, dev, stream, dq) if rank == 0 else None
+    e2e = None
+    if rank == 0 and not args.no_e2e:
+        e2e = (run_e2e(args, wlr, host_tables, batches_h, dev, stream, dq) if not big else
+               {"skipped": f"fp32 tables of {wlr.total_rows * wlr.d * 4 / 1e9:.0f} GB exceed the pinned-host budget"})
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -354,35 +409,64 @@ def _measured_hbm() -> float:
 def run_e2e(args, wl, host_tables, batches_h, dev, stream, dq) -> dict:
     """Same step through the public Python API, from and to pinned host memory:
     H2D of the tables and the lookup batch, quantize, look up, dequantize, and D2H
-    of the packed tables, the pooled output and the dequantized rows."""
+    of the packed tables, the pooled output and the dequantized rows. Table t's
+    upload, compute and download run on three streams, so they overlap with
+    table t-1's and t+1's."""
     import torch
     pin_x = [torch.from_numpy(h).pin_memory() for h in host_tables]
     pin_b = [(torch.from_numpy(i).pin_memory(), torch.from_numpy(o).pin_memory()) for i, o in batches_h]
     d = wl.d
     cld = dq._codes_ld(d)
     xs = [torch.empty_like(p, device=dev) for p in pin_x]
+    codes = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wl.rows]
+    sbs = [torch.empty((n, 2), dtype=torch.int16, device=dev) for n in wl.rows]
+    deqs = [torch.empty((n, d), dtype=torch.float32, device=dev) for n in wl.rows]
     h_codes = [torch.empty((n, cld), dtype=torch.uint8).pin_memory() for n in wl.rows]
     h_sb = [torch.empty((n, 2), dtype=torch.int16).pin_memory() for n in wl.rows]
     h_deq = [torch.empty((n, d), dtype=torch.float32).pin_memory() for n in wl.rows]
     h_out = torch.empty((wl.batch, wl.n_tables * d), dtype=torch.float32).pin_memory()
+    out = torch.empty((wl.batch, wl.n_tables * d), dtype=torch.float32, device=dev)
+    bi_d = torch.empty_like(pin_b[0][0], device=dev)
+    bo_d = torch.empty_like(pin_b[0][1], device=dev)
     h2d = sum(p.numel() * 4 for p in pin_x) + pin_b[0][0].numel() * 4 + pin_b[0][1].numel() * 4
-    d2h = sum(c.numel() + s.numel() * 2 + q.numel() * 4 for c, s, q in zip(h_codes, h_sb, h_deq)) + h_out.numel() * 4
+    d2h = sum(c.numel() + s_.numel() * 2 + q.numel() * 4 for c, s_, q in zip(h_codes, h_sb, h_deq)) + h_out.numel() * 4
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    order = sorted(range(wl.n_tables), key=lambda t: wl.rows[t])  # small tables first: short pipeline fill
 
     def step(k):
-        for p, x in zip(pin_x, xs):
-            x.copy_(p, non_blocking=True)
-        bi = pin_b[k % len(pin_b)][0].to(dev, non_blocking=True)
-        bo = pin_b[k % len(pin_b)][1].to(dev, non_blocking=True)
-        packed = []
-        for x, hc, hs in zip(xs, h_codes, h_sb):
-            c, s, _, _ = dq.quantize_rows(x, with_loss=False)
-            packed.append(dq.PackedTable(c, s))
-        out = dq.embbag(packed, d, bi, bo, wl.batch)
-        for (c, s), hc, hs, hq in zip(packed, h_codes, h_sb, h_deq):
-            hq.copy_(dq.dequantize_rows(c, s, d), non_blocking=True)
-            hc.copy_(c, non_blocking=True)
-            hs.copy_(s, non_blocking=True)
-        h_out.copy_(out, non_blocking=True)
+        bi, bo = pin_b[k % len(pin_b)]
+        prev = torch.cuda.Event()
+        prev.record(stream)      # the previous step's kernels and downloads are ordered before this
+        s_in.wait_event(prev)    # so uploads never overwrite buffers still being read
+        with torch.cuda.stream(s_in):
+            bi_d.copy_(bi, non_blocking=True)
+            bo_d.copy_(bo, non_blocking=True)
+        for t in order:
+            with torch.cuda.stream(s_in):
+                xs[t].copy_(pin_x[t], non_blocking=True)
+                up = torch.cuda.Event()
+                up.record(s_in)
+            stream.wait_event(up)
+            dq.dq_quantize_rows_int4(xs[t], xs[t].shape[0], d, d, codes[t], cld, sbs[t], None, None,
+                                     dq.DQ_MODE_GREEDY, None, stream)
+            dq.dq_dequantize_rows(codes[t], cld, sbs[t], codes[t].shape[0], d, deqs[t], d, stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            s_out.wait_event(done)
+            with torch.cuda.stream(s_out):
+                h_codes[t].copy_(codes[t], non_blocking=True)
+                h_sb[t].copy_(sbs[t], non_blocking=True)
+                h_deq[t].copy_(deqs[t], non_blocking=True)
+        dq.dq_embbag_int4_fwd([dq.PackedTable(c, s_) for c, s_ in zip(codes, sbs)], d, bi_d, bo_d,
+                              wl.batch, out, None, stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        s_out.wait_event(done)
+        with torch.cuda.stream(s_out):
+            h_out.copy_(out, non_blocking=True)
+        fin = torch.cuda.Event()
+        fin.record(s_out)
+        stream.wait_event(fin)
 
     steps = max(3, min(args.steps, 10))
     for k in range(2):
@@ -396,19 +480,22 @@ def run_e2e(args, wl, host_tables, batches_h, dev, stream, dq) -> dict:
     torch.cuda.synchronize(dev)
     ms = e0.elapsed_time(e1) / steps
     return {"value": wl.total_rows / (ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps,
+            "api": "int4_row_wise_b200.dq_* from pinned host buffers, upload/compute/download on 3 streams"}
 
 
 def main(argv=None) -> None:
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="kaggle", choices=W.WORKLOADS)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--ref-seconds", type=float, default=12.0,
                     help="seconds of oracle work in the CPU baseline (the reference arm spends ~10x this in all)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--streams", type=int, default=4, help="streams the per-table quantize launches spread over")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -221,19 +221,36 @@ __device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, in
         float2 Ca[H], Cb[H];
         if constexpr (FAST) {
             const Clip ca = clip_fast(lo_i1, hi_j, thr), cb = clip_fast(lo_i, hi_j1, thr);
-            bool hard = false;
-            errors_packed<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca, hard);
-            errors_packed<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb, hard);
-            if (hard) {
-                errors_fixup<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca);
-                errors_fixup<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb);
+            // each candidate is reduced as soon as its errors exist; a candidate with
+            // an element too close to a rounding tie (rare) is evaluated again with
+            // the IEEE fix-up
+            bool hard_a = false, hard_b = false;
+            errors_packed<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca, hard_a);
+            float la = tree_sum2<H>(Ca);
+            errors_packed<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb, hard_b);
+            float lb = tree_sum2<H>(Cb);
+            if (hard_a || hard_b) {
+                if (hard_a) {
+                    errors_packed<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca, hard_a);
+                    errors_fixup<H, HAS_Y, FULL>(xp, ca, kbase, d, Ca);
+                    la = tree_sum2<H>(Ca);
+                }
+                if (hard_b) {
+                    errors_packed<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb, hard_b);
+                    errors_fixup<H, HAS_Y, FULL>(xp, cb, kbase, d, Cb);
+                    lb = tree_sum2<H>(Cb);
+                }
             }
+            Ca[0].x = la;
+            Cb[0].x = lb;
         } else {
             errors_exact<H, HAS_Y, FULL>(xp, lo_i1, hi_j, kbase, d, Ca);
             errors_exact<H, HAS_Y, FULL>(xp, lo_i, hi_j1, kbase, d, Cb);
+            Ca[0].x = tree_sum2<H>(Ca);
+            Cb[0].x = tree_sum2<H>(Cb);
         }
-        const float la = row_sum<W>(tree_sum2<H>(Ca));
-        const float lb = row_sum<W>(tree_sum2<H>(Cb));
+        const float la = row_sum<W>(Ca[0].x);
+        const float lb = row_sum<W>(Cb[0].x);
         const bool right = lb < la;  // ties move left
         const float l = right ? lb : la;
         fi = right ? fi : fi + 1.0f;
@@ -252,7 +269,7 @@ __device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, in
 // One row per W lanes; M elements per lane; FULL: d == M * W (no padding);
 // VEC: 16-byte loads of x and vector stores of the codes are aligned.
 template <int M, int W, bool FULL, bool VEC>
-__global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, const int greedy)
+__global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, const int greedy)
 {
     constexpr bool HAS_Y = M > 1;
     constexpr int H = HAS_Y ? M / 2 : 1;
@@ -399,7 +416,7 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(const QuantArgs a, c
 template <int M, int W>
 cudaError_t launch_mw(const QuantArgs &a, int greedy, cudaStream_t stream)
 {
-    constexpr int kBlock = 256;
+    constexpr int kBlock = 128;   // measured: finer blocks shorten the last wave
     const int64_t threads = a.n * W;
     const int64_t grid = (threads + kBlock - 1) / kBlock;
     const bool full = a.d == M * W;

@@ -216,3 +216,44 @@ def random_packed_table(n_rows: int, d: int, seed: int, codes_ld: Optional[int] 
     bias = r.uniform(-0.2, 0.05, n_rows).astype(np.float16)
     sb = np.stack([scale.view(np.uint16), bias.view(np.uint16)], axis=1)
     return codes, np.ascontiguousarray(sb)
+
+
+# ---------------------------------------------------------------------------
+# parallel generation of large tables (identical values: same per-block keys)
+# ---------------------------------------------------------------------------
+def _fill_blocks(args):
+    from multiprocessing import shared_memory
+    name, shape, wl, t, blocks = args
+    shm = shared_memory.SharedMemory(name=name)
+    try:
+        out = np.ndarray(shape, dtype=np.float32, buffer=shm.buf)
+        for b in blocks:
+            blk = table_block(wl, t, b)
+            out[b * BLOCK_ROWS:b * BLOCK_ROWS + blk.shape[0]] = blk
+    finally:
+        del out
+        shm.close()
+    return len(blocks)
+
+
+class SharedTable:
+    """A table generated by a pool of processes into shared memory. `array` is
+    valid until close()."""
+
+    def __init__(self, wl: Workload, t: int, procs: Optional[int] = None):
+        import multiprocessing as mp
+        import os as _os
+        from multiprocessing import shared_memory
+        n, d = wl.rows[t], wl.d
+        self.shm = shared_memory.SharedMemory(create=True, size=max(n * d * 4, 4))
+        self.array = np.ndarray((n, d), dtype=np.float32, buffer=self.shm.buf)
+        nb = n_blocks(wl, t)
+        procs = procs or min(len(_os.sched_getaffinity(0)), 32)
+        chunks = [list(range(i, nb, procs)) for i in range(procs) if i < nb]
+        with mp.get_context("spawn").Pool(len(chunks)) as pool:
+            pool.map(_fill_blocks, [(self.shm.name, (n, d), wl, t, c) for c in chunks])
+
+    def close(self):
+        self.array = None
+        self.shm.close()
+        self.shm.unlink()
