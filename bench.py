@@ -399,6 +399,53 @@ def run_gpu(args, wl: W.Workload) -> None:
         dist.destroy_process_group()
 
 
+def run_lookup_only(args, wl: W.Workload) -> None:
+    """Times the lookup alone over random packed tables of the workload's sizes
+    (a few GB on the device at most, e.g. for profiling): K calls over n distinct
+    batches, each call's unique algorithmic bytes against the HBM peak."""
+    import torch
+    import int4_row_wise_b200 as dq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dq.load()
+    d = wl.d
+    cld = dq._codes_ld(d)
+    tables = []
+    for t, n in enumerate(wl.rows):
+        c, sb = W.random_packed_table(n, d, 500 + t, cld)
+        tables.append(dq.PackedTable(torch.from_numpy(c).to(dev), torch.from_numpy(sb.view(np.int16)).to(dev)))
+    n_batches = 4
+    bh = [W.lookup_batch(wl, batch_id=i) for i in range(n_batches)]
+    bd = [(torch.from_numpy(i).to(dev), torch.from_numpy(o).to(dev)) for i, o in bh]
+    nbytes = [_unique_bag_bytes(wl, i, o) for i, o in bh]
+    out = torch.empty((wl.batch, wl.n_tables * d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)  # 256 MB > L2: cold start per call
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for k in range(args.warmup):
+        dq.dq_embbag_int4_fwd(tables, d, bd[k % n_batches][0], bd[k % n_batches][1], wl.batch, out, None, stream)
+    torch.cuda.synchronize(dev)
+    for k in range(args.steps):
+        flush.zero_()
+        evs[k][0].record(stream)
+        dq.dq_embbag_int4_fwd(tables, d, bd[k % n_batches][0], bd[k % n_batches][1], wl.batch, out, None, stream)
+        evs[k][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    tot_bytes = sum(nbytes[k % n_batches] for k in range(args.steps))
+    gbs = tot_bytes / (sum(ms) / 1e3) / 1e9
+    hbm = _measured_hbm()
+    print(json.dumps({
+        "metric": "INT4 embedding-bag GB/s (unique algorithmic bytes, L2 flushed before each call)",
+        "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": sum(ms) / len(ms), "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": _workload_desc(wl), "tables": "random packed codes of the workload's table sizes",
+                   "l2": "256 MB flush written before every call"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "bytes_per_call": int(np.mean(nbytes))},
+        "gpu_launches": args.steps}), flush=True)
+
+
 def _measured_hbm() -> float:
     try:
         return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
@@ -495,6 +542,8 @@ def main(argv=None) -> None:
                     help="seconds of oracle work in the CPU baseline (the reference arm spends ~10x this in all)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (profiling runs)")
+    ap.add_argument("--lookup-only", action="store_true",
+                    help="time only the lookup, over random packed tables of the workload's sizes")
     ap.add_argument("--streams", type=int, default=4, help="streams the per-table quantize launches spread over")
     args = ap.parse_args(argv)
     if args.warmup < 3:
@@ -502,6 +551,8 @@ def main(argv=None) -> None:
     wl = W.workload(args.workload, seed=0)
     if args.impl == "reference":
         run_reference(args, wl)
+    elif args.lookup_only:
+        run_lookup_only(args, wl)
     else:
         run_gpu(args, wl)
 

@@ -208,8 +208,12 @@ def random_packed_table(n_rows: int, d: int, seed: int, codes_ld: Optional[int] 
     cb = (d + 1) // 2
     codes_ld = cb if codes_ld is None else codes_ld
     r = _rng(seed, 99, n_rows, _P_PACKED, d)
-    codes = np.zeros((n_rows, codes_ld), dtype=np.uint8)
-    codes[:, :cb] = r.integers(0, 256, (n_rows, cb), dtype=np.uint8)
+    raw = np.frombuffer(r.bytes(n_rows * cb), dtype=np.uint8).reshape(n_rows, cb)
+    if codes_ld == cb:
+        codes = raw.copy()
+    else:
+        codes = np.zeros((n_rows, codes_ld), dtype=np.uint8)
+        codes[:, :cb] = raw
     if d % 2:
         codes[:, cb - 1] &= 0x0F
     scale = r.uniform(1e-3, 2e-2, n_rows).astype(np.float16)

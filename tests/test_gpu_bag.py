@@ -56,7 +56,7 @@ def _gpu_bag(tabs, d, idx, off, B, flags=False):
 
 
 @pytest.mark.parametrize("d", [16, 32, 64, 128, 256, 512, 1024, 7, 48, 100])
-@pytest.mark.parametrize("pool", [(1, 1), (0, 3), (20, 80)])
+@pytest.mark.parametrize("pool", [(1, 1), (0, 3), (0, 10), (20, 80)])
 def test_bag_matches_oracle(cuda_device, d, pool):
     T, B = 3, 97
     rows = [500, 1000, 37]

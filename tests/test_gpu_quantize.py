@@ -82,6 +82,9 @@ def test_special_rows(cuda_device):
     rows.append((3.0 + 0.0625 * q[::-1]).astype(np.float32))
     rows.append(np.where(q % 2, 1e-39, 2e-39).astype(np.float32))  # subnormal inputs, tiny range
     rows.append(np.linspace(-1e30, 1e30, d).astype(np.float32))    # huge but fp32-finite range
+    r = np.random.default_rng(11)
+    rows.append((1000.0 + 1e-3 * r.standard_normal(d)).astype(np.float32))  # offset >> range: IEEE walk
+    rows.append((-3e4 + 0.05 * r.standard_normal(d)).astype(np.float32))
     x = np.stack(rows)
     g, o = assert_quant_parity(x)
     assert np.all(g[1][:6, 0] == 0) and np.all(g[0][:6] == 0)

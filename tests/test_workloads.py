@@ -57,3 +57,21 @@ def test_production_pooling_and_zipf_head():
     assert lens.min() >= 20 and lens.max() <= 80
     # Zipf(1.2): id 0 is the most frequent
     assert np.bincount(idx).argmax() == 0
+
+
+def test_shared_table_matches_serial_generation():
+    # the block-parallel generator (spawned processes) draws exactly the serial values
+    wl = W.workload("sweep-16")
+    st = W.SharedTable(wl, 0, procs=3)
+    try:
+        assert np.array_equal(st.array, W.table_rows(wl, 0))
+    finally:
+        st.close()
+
+
+def test_random_packed_table_layout():
+    codes, sb = W.random_packed_table(1000, 7, seed=1, codes_ld=16)
+    assert codes.shape == (1000, 16) and sb.shape == (1000, 2)
+    assert np.all(codes[:, 4:] == 0) and np.all(codes[:, 3] >> 4 == 0)
+    s = sb[:, 0].view(np.float16).astype(np.float32)
+    assert np.all(s > 0) and np.all(np.isfinite(sb.view(np.float16)))
