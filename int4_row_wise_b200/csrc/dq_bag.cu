@@ -100,8 +100,23 @@ __global__ void __launch_bounds__(256) dequant_generic_kernel(const DequantArgs 
 }
 
 // ---------------------------------------------------------------------------
-// embedding bag: G = d / E lanes per bag, E outputs (E/2 code bytes) per lane
+// embedding bag
+//
+// A bag is handled by G = EG * IS lanes: EG = d / E element groups (E outputs,
+// E/2 code bytes per lane: one 8- or 16-byte load per row) times IS id strides
+// (lane `is` takes ids p0 + is, p0 + is + IS, ...). Lanes are numbered
+// eg * IS + is, so the IS partial sums of an element group sit in neighbouring
+// lanes; a shuffle reduce-scatter then leaves lane `is` holding E / IS finished
+// sums, contiguous in the output row, and the bag's row is written as one
+// contiguous run. Short bags (average pooling < 4, e.g. one-hot lookups) use
+// IS = 1 and many bags per warp for memory-level parallelism; their rows are
+// staged through shared memory so that each warp store covers whole rows. The
+// kernel reads the id count (the last offset) to pick the layout, so the host
+// need not know the pooling.
 // ---------------------------------------------------------------------------
+constexpr int kBagThreads = 256;
+constexpr int kBagUnroll = 4;
+
 template <int E>
 struct CodeVec;
 template <>
@@ -118,94 +133,201 @@ struct CodeVec<32> {
     }
 };
 
-constexpr int kBagBlock = 256;
-constexpr int kBagUnroll = 4;
+// scale * 2^(-4k) for the nibble pairs (0,1), (2,3), (4,5->2), (6->3,7->4) of a word
+struct PairParams {
+    float2 s01, s23, s42, s34, bb;
+};
 
-template <int E>
-__global__ void __launch_bounds__(kBagBlock) embbag_kernel(const __grid_constant__ BagTables tabs,
-                                                           const BagArgs a)
+__device__ __forceinline__ PairParams pair_params(uint32_t sbw)
 {
-    using V = typename CodeVec<E>::T;
-    constexpr int NW = E / 8;
-    const int G = a.d / E;                      // lanes per bag, a power of two <= 32
-    const int bags_per_block = kBagBlock / G;
-    const int64_t total = (int64_t)a.T * a.batch;
-    const int64_t g0 = (int64_t)blockIdx.x * bags_per_block;
+    const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
+    const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
+    const float S1 = __fmul_rn(S, 0.0625f), S2 = __fmul_rn(S, 0.00390625f);
+    const float S3 = __fmul_rn(S, 0.000244140625f), S4 = __fmul_rn(S, 1.52587890625e-05f);
+    PairParams p;
+    p.s01 = make_float2(S, S1);
+    p.s23 = make_float2(S2, S3);
+    p.s42 = make_float2(S4, S2);
+    p.s34 = make_float2(S3, S4);
+    p.bb = make_float2(B, B);
+    return p;
+}
 
-    __shared__ int32_t soff[kBagBlock + 1];
-    for (int k = threadIdx.x; k <= bags_per_block; k += kBagBlock) {
-        const int64_t gi = g0 + k;
-        soff[k] = gi <= total ? __ldg(a.offsets + gi) : 0;
-    }
-    __syncthreads();
+__device__ __forceinline__ float magic_nibble(uint32_t w, int k)
+{
+    return __uint_as_float((w & (0xfu << (4 * k))) | 0x4B000000u);
+}
 
-    const int lb = threadIdx.x / G, sub = threadIdx.x - lb * G;
-    const int64_t g = g0 + lb;
-    if (g >= total)
-        return;
-    const int t = (int)(g / a.batch);
-    const int b = (int)(g - (int64_t)t * a.batch);
-    const int32_t n_ids = max(__ldg(a.offsets + total), 0);  // the id count
-    int32_t p = soff[lb];
-    int32_t p1 = soff[lb + 1];
-    if (p1 < p || p < 0 || p1 > n_ids) {
-        if (sub == 0)
-            raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
-        p = min(max(p, 0), n_ids);
-        p1 = max(min(p1, n_ids), p);
-    }
-    const uint8_t *codes = tabs.codes[t] + sub * (E / 2);
-    const uint32_t *sbp = reinterpret_cast<const uint32_t *>(tabs.scale_bias[t]);
-    const int64_t n_rows = tabs.n_rows[t];
-    const int64_t ld = tabs.codes_ld[t];
+// acc[0..7] += fma(q_k, scale, bias) for the 8 nibbles of w (packed f32x2 math).
+__device__ __forceinline__ void accumulate_word(uint32_t w, const PairParams &p, float2 (&acc)[4])
+{
+    const uint32_t hi = w >> 12;  // nibbles 5, 6, 7 -> bit positions 8, 12, 16
+    const float2 m23 = make_float2(-kTwo23, -kTwo23);
+    const float2 v01 = __fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23);
+    const float2 v23 = __fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23);
+    const float2 v45 = __fadd2_rn(make_float2(magic_nibble(w, 4), magic_nibble(hi, 2)), m23);
+    const float2 v67 = __fadd2_rn(make_float2(magic_nibble(hi, 3), magic_nibble(hi, 4)), m23);
+    acc[0] = __fadd2_rn(acc[0], __ffma2_rn(v01, p.s01, p.bb));
+    acc[1] = __fadd2_rn(acc[1], __ffma2_rn(v23, p.s23, p.bb));
+    acc[2] = __fadd2_rn(acc[2], __ffma2_rn(v45, p.s42, p.bb));
+    acc[3] = __fadd2_rn(acc[3], __ffma2_rn(v67, p.s34, p.bb));
+}
 
-    float acc[E];
+// Reduce-scatter of E sums over the IS id strides (lane bits 0..log2(IS)-1):
+// afterwards lane `is` holds elements [is * E/IS, (is+1) * E/IS) in acc[0 .. E/IS).
+template <int E, int IS>
+__device__ __forceinline__ void reduce_scatter(float (&acc)[E], int is)
+{
 #pragma unroll
-    for (int k = 0; k < E; ++k)
-        acc[k] = 0.0f;
-    bool bad = false;
-
-    for (; p < p1; p += kBagUnroll) {
-        int32_t id[kBagUnroll];
-        bool ok[kBagUnroll];
+    for (int j = 0, half = E / 2; (1 << j) < IS; ++j, half /= 2) {
+        // the highest stride bit splits first, so the kept chunk index is `is`
+        const int bitpos = 31 - __clz(IS) - 1 - j;
+        const bool upper = (is >> bitpos) & 1;
 #pragma unroll
-        for (int u = 0; u < kBagUnroll; ++u) {
-            id[u] = (p + u < p1) ? __ldg(a.indices + p + u) : 0;
-            ok[u] = (p + u < p1) && id[u] >= 0 && (int64_t)id[u] < n_rows;
-            bad |= (p + u < p1) && !ok[u];
-        }
-        V w[kBagUnroll];
-        uint32_t sbw[kBagUnroll];
-#pragma unroll
-        for (int u = 0; u < kBagUnroll; ++u) {
-            const int64_t r = ok[u] ? id[u] : 0;
-            if (ok[u]) {
-                w[u] = __ldg(reinterpret_cast<const V *>(codes + r * ld));
-                sbw[u] = __ldg(sbp + r);
+        for (int m = 0; m < E / 2; ++m) {
+            if (m < half) {
+                const float send = upper ? acc[m] : acc[m + half];
+                const float keep = upper ? acc[m + half] : acc[m];
+                acc[m] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, 1 << bitpos));
             }
         }
+    }
+}
+
+template <int E, int IS>
+__device__ __forceinline__ void bag_tiles(const BagTables &tabs, const BagArgs &a, int64_t total,
+                                          int32_t n_ids, float *stage)
+{
+    using V = typename CodeVec<E>::T;
+    constexpr int NW = E / 8;  // 32-bit code words per lane and row
+    const int EG = a.d / E;
+    const int G = EG * IS;     // lanes per bag, a power of two <= 32
+    const int bags_per_block = kBagThreads / G;
+    const int lg = threadIdx.x % G, lb = threadIdx.x / G;
+    const int is = lg % IS, eg = lg / IS;
+    const int lane = threadIdx.x & 31;
+
+    // T * batch + 1 <= INT32_MAX is checked on the host: 32-bit bag arithmetic
+    const uint32_t total32 = (uint32_t)total, batch = (uint32_t)a.batch;
+    for (uint32_t tile = blockIdx.x; (uint64_t)tile * bags_per_block < total32; tile += gridDim.x) {
+        const uint32_t g = tile * bags_per_block + lb;
+        const bool live = g < total32;
+        const int t = live ? (int)(g / batch) : 0;
+        const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
+        int32_t p = 0, p1 = 0;
+        if (live) {
+            p = __ldg(a.offsets + g);
+            p1 = __ldg(a.offsets + g + 1);
+            if (p1 < p || p < 0 || p1 > n_ids) {
+                if (lg == 0)
+                    raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
+                p = min(max(p, 0), n_ids);
+                p1 = max(min(p1, n_ids), p);
+            }
+        }
+        const uint8_t *codes = tabs.codes[t] + eg * (E / 2);
+        const uint32_t *sbp = reinterpret_cast<const uint32_t *>(tabs.scale_bias[t]);
+        const int64_t n_rows = tabs.n_rows[t];
+        const int64_t ld = tabs.codes_ld[t];
+
+        float2 acc2[E / 2];
 #pragma unroll
-        for (int u = 0; u < kBagUnroll; ++u) {
-            if (ok[u]) {
-                const RowParams prm = row_params(sbw[u]);
+        for (int k = 0; k < E / 2; ++k)
+            acc2[k] = make_float2(0.0f, 0.0f);
+        bool bad = false;
+        for (p += is; p < p1; p += IS * kBagUnroll) {
+            int32_t id[kBagUnroll];
+            bool ok[kBagUnroll];
 #pragma unroll
-                for (int i = 0; i < NW; ++i) {
-                    float x[8];
-                    decode_word(CodeVec<E>::word(w[u], i), prm, x);
+            for (int u = 0; u < kBagUnroll; ++u) {
+                const int32_t pu = p + u * IS;
+                id[u] = pu < p1 ? __ldg(a.indices + pu) : 0;
+                ok[u] = pu < p1 && id[u] >= 0 && (int64_t)id[u] < n_rows;
+                bad |= pu < p1 && !ok[u];
+            }
+            V w[kBagUnroll];
+            uint32_t sbw[kBagUnroll];
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
-                        acc[8 * i + k] = __fadd_rn(acc[8 * i + k], x[k]);
+            for (int u = 0; u < kBagUnroll; ++u) {
+                if (ok[u]) {
+                    w[u] = __ldg(reinterpret_cast<const V *>(codes + (int64_t)id[u] * ld));
+                    sbw[u] = __ldg(sbp + id[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < kBagUnroll; ++u) {
+                if (ok[u]) {
+                    const PairParams prm = pair_params(sbw[u]);
+#pragma unroll
+                    for (int i = 0; i < NW; ++i) {
+                        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
+                        accumulate_word(CodeVec<E>::word(w[u], i), prm, quad);
+                    }
                 }
             }
         }
-    }
-    if (bad && sub == 0)
-        raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+        if (bad)
+            raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
 
-    float4 *o = reinterpret_cast<float4 *>(a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d + sub * E);
+        float acc[E];
 #pragma unroll
-    for (int k = 0; k < E; k += 4)
-        o[k / 4] = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+        for (int k = 0; k < E / 2; ++k) {
+            acc[2 * k] = acc2[k].x;
+            acc[2 * k + 1] = acc2[k].y;
+        }
+        if constexpr (IS > 1) {
+            reduce_scatter<E, IS>(acc, is);
+            if (live) {
+                constexpr int C = E / IS;  // finished sums owned by this lane
+                float *o = a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d + eg * E + is * C;
+                if constexpr (C % 4 == 0) {
+#pragma unroll
+                    for (int k = 0; k < C; k += 4)
+                        reinterpret_cast<float4 *>(o)[k / 4] = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+                } else if constexpr (C == 2) {
+                    *reinterpret_cast<float2 *>(o) = make_float2(acc[0], acc[1]);
+                } else {
+                    o[0] = acc[0];
+                }
+            }
+        } else {
+            // stage the warp's rows (E + 4 floats per lane: conflict-free float4 writes)
+            float *st = stage + (threadIdx.x >> 5) * 32 * (E + 4);
+#pragma unroll
+            for (int k = 0; k < E; k += 4)
+                *reinterpret_cast<float4 *>(st + lane * (E + 4) + k) =
+                    make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+            __syncwarp();
+            // the warp's bags are consecutive: write each row as contiguous float4s; the
+            // first lane of each bag broadcasts its output row's address
+            const int bags_per_warp = 32 / EG;
+            float4 *row = reinterpret_cast<float4 *>(a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d);
+            const int q4_per_row = a.d / 4;
+            const uint32_t gw = tile * bags_per_block + (uint32_t)((threadIdx.x >> 5) * bags_per_warp);
+            for (int f = lane; f < bags_per_warp * q4_per_row; f += 32) {
+                const int bw = f / q4_per_row, c = f - bw * q4_per_row;
+                float4 *dst = reinterpret_cast<float4 *>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(row), bw * EG));
+                if (gw + bw < total32) {
+                    const int e0 = 4 * c, src_lane = bw * EG + e0 / E;
+                    dst[c] = *reinterpret_cast<const float4 *>(st + src_lane * (E + 4) + (e0 % E));
+                }
+            }
+            __syncwarp();
+        }
+    }
+}
+
+template <int E, int ISL>
+__global__ void __launch_bounds__(kBagThreads) embbag_kernel(const __grid_constant__ BagTables tabs,
+                                                             const BagArgs a)
+{
+    __shared__ __align__(16) float stage[(kBagThreads / 32) * 32 * (E + 4)];
+    const int64_t total = (int64_t)a.T * a.batch;
+    const int32_t n_ids = max(__ldg(a.offsets + total), 0);
+    if (ISL > 1 && (int64_t)n_ids >= 4 * total)   // average pooling >= 4: split ids over lanes
+        bag_tiles<E, ISL>(tabs, a, total, n_ids, stage);
+    else
+        bag_tiles<E, 1>(tabs, a, total, n_ids, stage);
 }
 
 // any d, any alignment: one warp per bag, lanes stride over the elements
@@ -275,7 +397,7 @@ cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t st
     return cudaGetLastError();
 }
 
-cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int /*num_sms*/, cudaStream_t stream)
+cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream)
 {
     const int64_t total = (int64_t)a.T * a.batch;
     int E = 0;
@@ -288,13 +410,22 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int /*num_sms
         fast = tabs.codes_ld[t] % (E / 2) == 0 && (reinterpret_cast<uintptr_t>(tabs.codes[t]) % (E / 2)) == 0 &&
                (reinterpret_cast<uintptr_t>(tabs.scale_bias[t]) & 3) == 0;
     if (fast) {
-        const int G = a.d / E;
-        const int bags_per_block = kBagBlock / G;
-        const int64_t grid = (total + bags_per_block - 1) / bags_per_block;
+        const int EG = a.d / E;
+        const int isl = E == 16 || EG <= 4 ? 8 : EG == 8 ? 4 : EG == 16 ? 2 : 1;
+        const int bags_per_block = kBagThreads / (EG * isl);  // the smaller (long-bag) tile
+        const int64_t tiles = (total + bags_per_block - 1) / bags_per_block;
+        const int64_t cap = (int64_t)num_sms * 8;       // grid-stride beyond one resident wave
+        const unsigned grid = (unsigned)(tiles < cap ? tiles : cap);
         if (E == 16)
-            embbag_kernel<16><<<(unsigned)grid, kBagBlock, 0, stream>>>(tabs, a);
+            embbag_kernel<16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+        else if (EG <= 4)
+            embbag_kernel<32, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+        else if (EG == 8)
+            embbag_kernel<32, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+        else if (EG == 16)
+            embbag_kernel<32, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);
         else
-            embbag_kernel<32><<<(unsigned)grid, kBagBlock, 0, stream>>>(tabs, a);
+            embbag_kernel<32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);
     } else {
         const int64_t grid = (total * 32 + 255) / 256;
         embbag_generic_kernel<<<(unsigned)grid, 256, 0, stream>>>(tabs, a);
