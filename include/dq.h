@@ -79,7 +79,7 @@ typedef struct dq_table {
     const uint8_t *codes;
     const uint16_t *scale_bias;
     int64_t n_rows;
-    int64_t codes_ld;   /* bytes between rows, >= (d + 1) / 2 */
+    int64_t codes_ld;   /* bytes between rows, in [(d + 1) / 2, 2^31) */
 } dq_table;
 
 /*

@@ -152,7 +152,10 @@ def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, o
     arr = (_Table * max(len(tables), 1))()
     for t, tab in enumerate(tables):
         codes, sb = tab[0], tab[1]
-        ld = int(codes.stride(0)) if codes.dim() == 2 else 0
+        if codes.dim() != 2:
+            raise DqError(DQ_ERR_INVALID_ARG, "table codes must be a [n_rows, codes_ld] tensor")
+        # a table of 0 or 1 rows has no meaningful row stride: its row width is the stride
+        ld = int(codes.stride(0)) if codes.shape[0] > 1 else int(codes.shape[1])
         arr[t] = _Table(_ptr(codes), _ptr(sb), int(codes.shape[0]), ld)
     st = load().dq_embbag_int4_fwd(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
                                    _ptr(offsets), batch, _ptr(out), _ptr(d_flags), _stream(stream))

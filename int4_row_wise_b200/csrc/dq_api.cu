@@ -152,8 +152,8 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
         const dq_table &tb = tables[t];
         if (tb.n_rows < 0)
             return fail(DQ_ERR_INVALID_ARG, "tables[%d].n_rows = %lld < 0", t, (long long)tb.n_rows);
-        if (tb.codes_ld < (d + 1) / 2)
-            return fail(DQ_ERR_INVALID_ARG, "tables[%d].codes_ld = %lld < (d+1)/2 = %d", t,
+        if (tb.codes_ld < (d + 1) / 2 || tb.codes_ld > INT32_MAX)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].codes_ld = %lld outside [(d+1)/2 = %d, 2^31)", t,
                         (long long)tb.codes_ld, (d + 1) / 2);
         if (tb.n_rows > 0 && (!tb.codes || !tb.scale_bias))
             return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codes and scale_bias must be non-NULL", t);

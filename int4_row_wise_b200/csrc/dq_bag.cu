@@ -115,7 +115,6 @@ __global__ void __launch_bounds__(256) dequant_generic_kernel(const DequantArgs 
 // need not know the pooling.
 // ---------------------------------------------------------------------------
 constexpr int kBagThreads = 256;
-constexpr int kBagUnroll = 4;
 
 template <int E>
 struct CodeVec;
@@ -194,126 +193,229 @@ __device__ __forceinline__ void reduce_scatter(float (&acc)[E], int is)
     }
 }
 
-template <int E, int IS>
-__device__ __forceinline__ void bag_tiles(const BagTables &tabs, const BagArgs &a, int64_t total,
-                                          int32_t n_ids, float *stage)
+// One table's view for the bag currently handled by a lane.
+struct TableView {
+    const uint8_t *codes;     // this lane's element group within row 0
+    const uint32_t *sb;       // {scale, bias} of row 0 as one 32-bit word
+    uint32_t n_rows;          // rows addressable by an int32 id
+    uint32_t ld;              // code bytes between rows
+};
+
+__device__ __forceinline__ TableView table_view(const BagTables &tabs, int t, int eg, int E)
+{
+    TableView v;
+    v.codes = tabs.codes[t] + eg * (E / 2);
+    v.sb = reinterpret_cast<const uint32_t *>(tabs.scale_bias[t]);
+    v.n_rows = (uint32_t)min(tabs.n_rows[t], (int64_t)0x80000000LL);
+    v.ld = (uint32_t)tabs.codes_ld[t];
+    return v;
+}
+
+// acc += the E dequantized values of code vector w with packed scale/bias sbw
+template <int E>
+__device__ __forceinline__ void accumulate_row(const typename CodeVec<E>::T &w, uint32_t sbw,
+                                               float2 (&acc2)[E / 2])
+{
+    const PairParams prm = pair_params(sbw);
+#pragma unroll
+    for (int i = 0; i < E / 8; ++i) {
+        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
+        accumulate_word(CodeVec<E>::word(w, i), prm, quad);
+    }
+}
+
+// Sums the ids at positions q, q + step, ... < p1 into acc2 (groups of 4 loads in
+// flight, then single ids). Out-of-range ids are skipped and reported in `bad`.
+template <int E>
+__device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indices, int32_t q, int32_t p1,
+                                               int step, const TableView &tv, float2 (&acc2)[E / 2],
+                                               bool &bad)
 {
     using V = typename CodeVec<E>::T;
-    constexpr int NW = E / 8;  // 32-bit code words per lane and row
+    for (; q + 3 * step < p1; q += 4 * step) {
+        uint32_t id[4];
+        bool ok[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            id[u] = (uint32_t)__ldg(indices + q + u * step);
+            ok[u] = id[u] < tv.n_rows;
+            bad |= !ok[u];
+        }
+        V w[4];
+        uint32_t sbw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if (ok[u]) {
+                w[u] = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id[u] * tv.ld));
+                sbw[u] = __ldg(tv.sb + id[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (ok[u])
+                accumulate_row<E>(w[u], sbw[u], acc2);
+    }
+    for (; q < p1; q += step) {
+        const uint32_t id = (uint32_t)__ldg(indices + q);
+        if (id < tv.n_rows) {
+            accumulate_row<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)),
+                              __ldg(tv.sb + id), acc2);
+        } else {
+            bad = true;
+        }
+    }
+}
+
+__device__ __forceinline__ void clamp_bag(int32_t &p, int32_t &p1, int32_t n_ids, bool report, uint32_t *flags)
+{
+    if (p1 < p || p < 0 || p1 > n_ids) {
+        if (report)
+            raise_flag(flags, DQ_FLAG_BAD_OFFSETS);
+        p = min(max(p, 0), n_ids);
+        p1 = max(min(p1, n_ids), p);
+    }
+}
+
+// Long bags: IS id strides per element group, reduce-scatter, contiguous row stores.
+template <int E, int IS>
+__device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagArgs &a, uint32_t total,
+                                               int32_t n_ids)
+{
     const int EG = a.d / E;
     const int G = EG * IS;     // lanes per bag, a power of two <= 32
-    const int bags_per_block = kBagThreads / G;
+    const uint32_t bags_per_block = kBagThreads / G;
     const int lg = threadIdx.x % G, lb = threadIdx.x / G;
     const int is = lg % IS, eg = lg / IS;
-    const int lane = threadIdx.x & 31;
-
-    // T * batch + 1 <= INT32_MAX is checked on the host: 32-bit bag arithmetic
-    const uint32_t total32 = (uint32_t)total, batch = (uint32_t)a.batch;
-    for (uint32_t tile = blockIdx.x; (uint64_t)tile * bags_per_block < total32; tile += gridDim.x) {
+    const uint32_t batch = (uint32_t)a.batch;
+    for (uint32_t tile = blockIdx.x; (uint64_t)tile * bags_per_block < total; tile += gridDim.x) {
         const uint32_t g = tile * bags_per_block + lb;
-        const bool live = g < total32;
+        const bool live = g < total;
         const int t = live ? (int)(g / batch) : 0;
         const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
         int32_t p = 0, p1 = 0;
         if (live) {
             p = __ldg(a.offsets + g);
             p1 = __ldg(a.offsets + g + 1);
-            if (p1 < p || p < 0 || p1 > n_ids) {
-                if (lg == 0)
-                    raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
-                p = min(max(p, 0), n_ids);
-                p1 = max(min(p1, n_ids), p);
-            }
+            clamp_bag(p, p1, n_ids, lg == 0, a.flags);
         }
-        const uint8_t *codes = tabs.codes[t] + eg * (E / 2);
-        const uint32_t *sbp = reinterpret_cast<const uint32_t *>(tabs.scale_bias[t]);
-        const int64_t n_rows = tabs.n_rows[t];
-        const int64_t ld = tabs.codes_ld[t];
-
+        const TableView tv = table_view(tabs, t, eg, E);
         float2 acc2[E / 2];
 #pragma unroll
         for (int k = 0; k < E / 2; ++k)
             acc2[k] = make_float2(0.0f, 0.0f);
         bool bad = false;
-        for (p += is; p < p1; p += IS * kBagUnroll) {
-            int32_t id[kBagUnroll];
-            bool ok[kBagUnroll];
-#pragma unroll
-            for (int u = 0; u < kBagUnroll; ++u) {
-                const int32_t pu = p + u * IS;
-                id[u] = pu < p1 ? __ldg(a.indices + pu) : 0;
-                ok[u] = pu < p1 && id[u] >= 0 && (int64_t)id[u] < n_rows;
-                bad |= pu < p1 && !ok[u];
-            }
-            V w[kBagUnroll];
-            uint32_t sbw[kBagUnroll];
-#pragma unroll
-            for (int u = 0; u < kBagUnroll; ++u) {
-                if (ok[u]) {
-                    w[u] = __ldg(reinterpret_cast<const V *>(codes + (int64_t)id[u] * ld));
-                    sbw[u] = __ldg(sbp + id[u]);
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < kBagUnroll; ++u) {
-                if (ok[u]) {
-                    const PairParams prm = pair_params(sbw[u]);
-#pragma unroll
-                    for (int i = 0; i < NW; ++i) {
-                        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
-                        accumulate_word(CodeVec<E>::word(w[u], i), prm, quad);
-                    }
-                }
-            }
-        }
+        accumulate_ids<E>(a.indices, p + is, p1, IS, tv, acc2, bad);
         if (bad)
             raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
-
         float acc[E];
 #pragma unroll
         for (int k = 0; k < E / 2; ++k) {
             acc[2 * k] = acc2[k].x;
             acc[2 * k + 1] = acc2[k].y;
         }
-        if constexpr (IS > 1) {
-            reduce_scatter<E, IS>(acc, is);
-            if (live) {
-                constexpr int C = E / IS;  // finished sums owned by this lane
-                float *o = a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d + eg * E + is * C;
-                if constexpr (C % 4 == 0) {
+        reduce_scatter<E, IS>(acc, is);
+        if (live) {
+            constexpr int C = E / IS;  // finished sums owned by this lane
+            float *o = a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d + eg * E + is * C;
+            if constexpr (C % 4 == 0) {
 #pragma unroll
-                    for (int k = 0; k < C; k += 4)
-                        reinterpret_cast<float4 *>(o)[k / 4] = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
-                } else if constexpr (C == 2) {
-                    *reinterpret_cast<float2 *>(o) = make_float2(acc[0], acc[1]);
-                } else {
-                    o[0] = acc[0];
-                }
+                for (int k = 0; k < C; k += 4)
+                    reinterpret_cast<float4 *>(o)[k / 4] = make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
+            } else if constexpr (C == 2) {
+                *reinterpret_cast<float2 *>(o) = make_float2(acc[0], acc[1]);
+            } else {
+                o[0] = acc[0];
             }
-        } else {
-            // stage the warp's rows (E + 4 floats per lane: conflict-free float4 writes)
-            float *st = stage + (threadIdx.x >> 5) * 32 * (E + 4);
-#pragma unroll
-            for (int k = 0; k < E; k += 4)
-                *reinterpret_cast<float4 *>(st + lane * (E + 4) + k) =
-                    make_float4(acc[k], acc[k + 1], acc[k + 2], acc[k + 3]);
-            __syncwarp();
-            // the warp's bags are consecutive: write each row as contiguous float4s; the
-            // first lane of each bag broadcasts its output row's address
-            const int bags_per_warp = 32 / EG;
-            float4 *row = reinterpret_cast<float4 *>(a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d);
-            const int q4_per_row = a.d / 4;
-            const uint32_t gw = tile * bags_per_block + (uint32_t)((threadIdx.x >> 5) * bags_per_warp);
-            for (int f = lane; f < bags_per_warp * q4_per_row; f += 32) {
-                const int bw = f / q4_per_row, c = f - bw * q4_per_row;
-                float4 *dst = reinterpret_cast<float4 *>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(row), bw * EG));
-                if (gw + bw < total32) {
-                    const int e0 = 4 * c, src_lane = bw * EG + e0 / E;
-                    dst[c] = *reinterpret_cast<const float4 *>(st + src_lane * (E + 4) + (e0 % E));
-                }
-            }
-            __syncwarp();
         }
+    }
+}
+
+// Short bags (one-hot lookups): many bags per warp, one lane per element group.
+// A tile's offsets and the id at the bag's own position (where a one-hot bag keeps
+// its id) are loaded one tile ahead, so only the row load waits on the loop.
+// Rows are staged in shared memory and written back as whole contiguous rows.
+template <int E>
+__device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const BagArgs &a, uint32_t total,
+                                                int32_t n_ids, float *stage)
+{
+    using V = typename CodeVec<E>::T;
+    const int EG = a.d / E;
+    const uint32_t bags_per_block = kBagThreads / EG;
+    const int lb = threadIdx.x / EG, eg = threadIdx.x % EG;
+    const int lane = threadIdx.x & 31;
+    const int bags_per_warp = 32 / EG;
+    const int q4_shift = 31 - __clz(a.d / 4);   // d / 4 float4 per row, a power of two
+    const uint32_t batch = (uint32_t)a.batch;
+    float *st = stage + (threadIdx.x >> 5) * 32 * (E + 4);
+
+    uint32_t tile = blockIdx.x;
+    int32_t nx_p = 0, nx_p1 = 0, nx_id = 0;
+    {
+        const uint32_t g = tile * bags_per_block + lb;
+        if ((uint64_t)tile * bags_per_block < total && g < total) {
+            nx_p = __ldg(a.offsets + g);
+            nx_p1 = __ldg(a.offsets + g + 1);
+            nx_id = (int32_t)g < n_ids ? __ldg(a.indices + g) : 0;
+        }
+    }
+    for (; (uint64_t)tile * bags_per_block < total; tile += gridDim.x) {
+        const uint32_t g = tile * bags_per_block + lb;
+        const bool live = g < total;
+        int32_t p = nx_p, p1 = nx_p1;
+        const int32_t spec_id = nx_id;
+        {   // the next tile's offsets and speculative ids
+            const uint64_t tn = (uint64_t)tile + gridDim.x;
+            const uint64_t gn = tn * bags_per_block + lb;
+            if (gn < total) {
+                nx_p = __ldg(a.offsets + gn);
+                nx_p1 = __ldg(a.offsets + gn + 1);
+                nx_id = (int64_t)gn < n_ids ? __ldg(a.indices + gn) : 0;
+            }
+        }
+        const int t = live ? (int)(g / batch) : 0;
+        const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
+        if (live)
+            clamp_bag(p, p1, n_ids, eg == 0, a.flags);
+        else
+            p = p1 = 0;
+        const TableView tv = table_view(tabs, t, eg, E);
+        float2 acc2[E / 2];
+#pragma unroll
+        for (int k = 0; k < E / 2; ++k)
+            acc2[k] = make_float2(0.0f, 0.0f);
+        bool bad = false;
+        if (p1 == p + 1) {  // one id: the speculative load holds it when it sits at position g
+            const uint32_t id = (uint32_t)(p == (int32_t)g ? spec_id : __ldg(a.indices + p));
+            if (id < tv.n_rows)
+                accumulate_row<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)),
+                                  __ldg(tv.sb + id), acc2);
+            else
+                bad = true;
+        } else if (p1 > p) {
+            accumulate_ids<E>(a.indices, p, p1, 1, tv, acc2, bad);
+        }
+        if (bad)
+            raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+
+        // stage the warp's rows (E + 4 floats per lane: conflict-free float4 writes)
+#pragma unroll
+        for (int k = 0; k < E / 2; k += 2)
+            *reinterpret_cast<float4 *>(st + lane * (E + 4) + 2 * k) =
+                make_float4(acc2[k].x, acc2[k].y, acc2[k + 1].x, acc2[k + 1].y);
+        __syncwarp();
+        // the warp's bags are consecutive: write each row as contiguous float4s; the
+        // first lane of each bag broadcasts its output row's address
+        float4 *row = reinterpret_cast<float4 *>(a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d);
+        const uint32_t gw = tile * bags_per_block + (uint32_t)((threadIdx.x >> 5) * bags_per_warp);
+        for (int f = lane; f < 8 * E; f += 32) {   // the warp's 32 * E / 4 float4
+            const int bw = f >> q4_shift, c = f & ((1 << q4_shift) - 1);
+            float4 *dst = reinterpret_cast<float4 *>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(row), bw * EG));
+            if (gw + bw < total) {
+                const int e0 = 4 * c;
+                dst[c] = *reinterpret_cast<const float4 *>(st + (bw * EG + e0 / E) * (E + 4) + (e0 % E));
+            }
+        }
+        __syncwarp();
     }
 }
 
@@ -325,9 +427,9 @@ __global__ void __launch_bounds__(kBagThreads) embbag_kernel(const __grid_consta
     const int64_t total = (int64_t)a.T * a.batch;
     const int32_t n_ids = max(__ldg(a.offsets + total), 0);
     if (ISL > 1 && (int64_t)n_ids >= 4 * total)   // average pooling >= 4: split ids over lanes
-        bag_tiles<E, ISL>(tabs, a, total, n_ids, stage);
+        bag_tiles_long<E, ISL>(tabs, a, (uint32_t)total, n_ids);
     else
-        bag_tiles<E, 1>(tabs, a, total, n_ids, stage);
+        bag_tiles_short<E>(tabs, a, (uint32_t)total, n_ids, stage);
 }
 
 // any d, any alignment: one warp per bag, lanes stride over the elements

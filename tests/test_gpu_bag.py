@@ -113,3 +113,32 @@ def test_workload_batches_on_random_tables(cuda_device, name):
     bag_tolerance_check(got, ref, mag)
     if wl.pooling == (1, 1):
         assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_bag_into_empty_table_skips_every_id(cuda_device):
+    d, B = 64, 8
+    full = _packed(50, d, 1)
+    empty = (np.zeros((0, 32), np.uint8), np.zeros((0, 2), np.uint16))
+    idx = np.array([0, 1, 2, 3, 4, 5, 6, 7, 0, 1, 2, 3, 4, 5, 6, 7], np.int32)
+    off = np.arange(0, 17, 1, dtype=np.int32)  # 2 tables x 8 one-id bags
+    got, fl = _gpu_bag([full, empty], d, idx, off, B, flags=True)
+    ref, mag, skipped = oracle.embbag([full, empty], d, idx, off, B, with_abs_sum=True)
+    assert skipped == 8 and fl & dq.DQ_FLAG_BAD_INDEX
+    assert np.all(got[:, d:] == 0)
+    assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_injected_launch_failure_raises(cuda_device, monkeypatch):
+    x = torch.zeros((10, 16), dtype=torch.float32, device="cuda")
+    codes = torch.full((10, 8), 7, dtype=torch.uint8, device="cuda")
+    sb = torch.zeros((10, 2), dtype=torch.int16, device="cuda")
+    monkeypatch.setenv("DQ_FAULT_INJECT", "launch")
+    with pytest.raises(dq.DqError) as ei:
+        dq.dq_quantize_rows_int4(x, 10, 16, 16, codes, 8, sb)
+    assert ei.value.status == dq.DQ_ERR_CUDA and "injected" in str(ei.value)
+    torch.cuda.synchronize()
+    assert torch.all(codes == 7)  # nothing was launched
+    monkeypatch.delenv("DQ_FAULT_INJECT")
+    dq.dq_quantize_rows_int4(x, 10, 16, 16, codes, 8, sb)
+    torch.cuda.synchronize()
+    assert torch.all(codes == 0)
