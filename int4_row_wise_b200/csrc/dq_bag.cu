@@ -503,7 +503,7 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, 
 {
     const int64_t total = (int64_t)a.T * a.batch;
     int E = 0;
-    if (a.d == 16)
+    if (a.d % 16 == 0 && a.d / 16 <= 32 && ((a.d / 16) & (a.d / 16 - 1)) == 0)
         E = 16;
     else if (a.d % 32 == 0 && a.d / 32 <= 32 && ((a.d / 32) & (a.d / 32 - 1)) == 0)
         E = 32;
@@ -513,21 +513,19 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, 
                (reinterpret_cast<uintptr_t>(tabs.scale_bias[t]) & 3) == 0;
     if (fast) {
         const int EG = a.d / E;
-        const int isl = E == 16 || EG <= 4 ? 8 : EG == 8 ? 4 : EG == 16 ? 2 : 1;
-        const int bags_per_block = kBagThreads / (EG * isl);  // the smaller (long-bag) tile
+        const int isl = EG <= 4 ? 8 : EG == 8 ? 4 : EG == 16 ? 2 : 1;
+        const int bags_per_block = kBagThreads / (EG * isl);
         const int64_t tiles = (total + bags_per_block - 1) / bags_per_block;
-        const int64_t cap = (int64_t)num_sms * 8;       // grid-stride beyond one resident wave
+        const int64_t cap = (int64_t)num_sms * 8;
         const unsigned grid = (unsigned)(tiles < cap ? tiles : cap);
-        if (E == 16)
-            embbag_kernel<16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        else if (EG <= 4)
-            embbag_kernel<32, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        else if (EG == 8)
-            embbag_kernel<32, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        else if (EG == 16)
-            embbag_kernel<32, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        else
+        if (E == 16) {
+            if (isl == 8) embbag_kernel<16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+            else if (isl == 4) embbag_kernel<16, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+            else if (isl == 2) embbag_kernel<16, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+            else embbag_kernel<16, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+        } else {
             embbag_kernel<32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);
+        }
     } else {
         const int64_t grid = (total * 32 + 255) / 256;
         embbag_generic_kernel<<<(unsigned)grid, 256, 0, stream>>>(tabs, a);

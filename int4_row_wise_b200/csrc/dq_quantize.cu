@@ -103,6 +103,7 @@ struct Clip {
     float lo, s;      // bias and scale of the candidate quantizer
     float r, nlr;     // rcp(hi - lo) and -RN(lo * r): u = sat(fma(x, r, nlr))
     float thr;        // |15u - q| above thr: too close to a rounding tie, recompute
+    uint32_t c_lo, c_span;  // e^2 with bits in [c_lo, c_lo + c_span): near a tie
 };
 
 __device__ __forceinline__ Clip clip_fast(float lo, float hi, float thr)
@@ -114,6 +115,14 @@ __device__ __forceinline__ Clip clip_fast(float lo, float hi, float thr)
     c.nlr = __fmul_rn(-lo, c.r);
     c.s = div15(w);
     c.thr = thr;
+    // |e| / s within b of 1/2 where b = 0.5 - thr (the tie margin) widened for the
+    // rounding of xhat and e: e^2 in s^2 [(1/2 - b')^2, (1/2 + b')^2]
+    const float b = __fmaf_rn(2.0f, 0.5f - thr, 1.52587890625e-05f);
+    const float s2 = __fmul_rn(c.s, c.s);
+    const float lo_c = __fmul_rn(s2, __fmaf_rn(-b, 1.0f - b, 0.25f) * 0.999999f);
+    const float hi_c = __fmul_rn(s2, __fmaf_rn(b, 1.0f + b, 0.25f) * 1.000001f);
+    c.c_lo = __float_as_uint(lo_c);
+    c.c_span = __float_as_uint(hi_c) - c.c_lo;
     return c;
 }
 
@@ -144,13 +153,12 @@ __device__ __forceinline__ void errors_packed(const float2 (&xp)[H], const Clip 
         const float2 U = make_float2(fma_sat(xp[h].x, c.r, c.nlr), fma_sat(xp[h].y, c.r, c.nlr));
         const float2 Z = __ffma2_rn(U, k15, kmag);     // kMagic + rint(15u)
         const float2 NQ = __ffma2_rn(Z, km1, kmag);    // -q, exact
-        const float2 DD = __ffma2_rn(U, k15, NQ);      // 15u - q
-        hard |= fabsf(DD.x) > c.thr;
-        if (HAS_Y)
-            hard |= fabsf(DD.y) > c.thr;
         const float2 XH = __ffma2_rn(NQ, ns2, lo2);    // q*s + lo, rounded once
         const float2 E = __ffma2_rn(XH, km1, xp[h]);   // x - xhat
         C[h] = __fmul2_rn(E, E);
+        hard |= __float_as_uint(C[h].x) - c.c_lo < c.c_span;
+        if (HAS_Y)
+            hard |= __float_as_uint(C[h].y) - c.c_lo < c.c_span;
         if (!valid_x<H, HAS_Y, FULL>(kbase, h, d))
             C[h].x = 0.0f;
         if (!valid_y<H, HAS_Y, FULL>(kbase, h, d))
@@ -173,9 +181,9 @@ __device__ __forceinline__ void errors_fixup(const float2 (&xp)[H], const Clip &
 {
 #pragma unroll
     for (int h = 0; h < H; ++h) {
-        if (valid_x<H, HAS_Y, FULL>(kbase, h, d) && fabsf(tie_distance(xp[h].x, c)) > c.thr)
+        if (valid_x<H, HAS_Y, FULL>(kbase, h, d) && __float_as_uint(C[h].x) - c.c_lo < c.c_span)
             C[h].x = sq_err_exact(xp[h].x, c.lo, c.s);
-        if (valid_y<H, HAS_Y, FULL>(kbase, h, d) && fabsf(tie_distance(xp[h].y, c)) > c.thr)
+        if (valid_y<H, HAS_Y, FULL>(kbase, h, d) && __float_as_uint(C[h].y) - c.c_lo < c.c_span)
             C[h].y = sq_err_exact(xp[h].y, c.lo, c.s);
     }
 }
