@@ -330,15 +330,57 @@ __device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagA
     }
 }
 
-// Short bags (one-hot lookups): many bags per warp, one lane per element group.
-// A tile's offsets and the id at the bag's own position (where a one-hot bag keeps
-// its id) are loaded one tile ahead, so only the row load waits on the loop.
+// What a lane fetches ahead for one bag of the short-bag layout: its offsets and
+// the id at the bag's own position g (where a one-hot bag keeps its id).
+struct ShortAhead {
+    int32_t p, p1, id;
+};
+
+__device__ __forceinline__ ShortAhead short_ahead(const BagArgs &a, uint64_t g, uint32_t total, int32_t n_ids)
+{
+    ShortAhead s{0, 0, 0};
+    if (g < total) {
+        s.p = __ldg(a.offsets + g);
+        s.p1 = __ldg(a.offsets + g + 1);
+        s.id = (int64_t)g < n_ids ? __ldg(a.indices + g) : 0;
+    }
+    return s;
+}
+
+// The row of a one-hot bag whose id sits at its own position, loaded one tile ahead.
+template <int E>
+struct ShortRow {
+    typename CodeVec<E>::T w;
+    uint32_t sb;
+    bool ready;
+};
+
+template <int E>
+__device__ __forceinline__ ShortRow<E> short_row(const BagTables &tabs, const BagArgs &a, const ShortAhead &s,
+                                                 uint64_t g, uint32_t total, int32_t n_ids, int eg)
+{
+    ShortRow<E> r;
+    r.ready = false;
+    if (g < total && (int64_t)s.p == (int64_t)g && s.p1 == s.p + 1 && s.p1 <= n_ids) {
+        const int t = (int)((uint32_t)g / (uint32_t)a.batch);
+        const TableView tv = table_view(tabs, t, eg, E);
+        if ((uint32_t)s.id < tv.n_rows) {
+            r.w = __ldg(reinterpret_cast<const typename CodeVec<E>::T *>(tv.codes + (uint64_t)(uint32_t)s.id * tv.ld));
+            r.sb = __ldg(tv.sb + (uint32_t)s.id);
+            r.ready = true;
+        }
+    }
+    return r;
+}
+
+// Short bags (one-hot lookups): many bags per warp, one lane per element group. A
+// two-stage pipeline keeps loads in flight across tiles: the offsets and the id at
+// the bag's own position two tiles ahead, the row of a one-hot bag one tile ahead.
 // Rows are staged in shared memory and written back as whole contiguous rows.
 template <int E>
 __device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const BagArgs &a, uint32_t total,
                                                 int32_t n_ids, float *stage)
 {
-    using V = typename CodeVec<E>::T;
     const int EG = a.d / E;
     const uint32_t bags_per_block = kBagThreads / EG;
     const int lb = threadIdx.x / EG, eg = threadIdx.x % EG;
@@ -346,34 +388,26 @@ __device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const Bag
     const int bags_per_warp = 32 / EG;
     const int q4_shift = 31 - __clz(a.d / 4);   // d / 4 float4 per row, a power of two
     const uint32_t batch = (uint32_t)a.batch;
+    const uint64_t gstride = (uint64_t)gridDim.x * bags_per_block;
     float *st = stage + (threadIdx.x >> 5) * 32 * (E + 4);
 
     uint32_t tile = blockIdx.x;
-    int32_t nx_p = 0, nx_p1 = 0, nx_id = 0;
-    {
-        const uint32_t g = tile * bags_per_block + lb;
-        if ((uint64_t)tile * bags_per_block < total && g < total) {
-            nx_p = __ldg(a.offsets + g);
-            nx_p1 = __ldg(a.offsets + g + 1);
-            nx_id = (int32_t)g < n_ids ? __ldg(a.indices + g) : 0;
-        }
-    }
+    const uint64_t g0 = (uint64_t)tile * bags_per_block + lb;
+    ShortAhead ahead1 = short_ahead(a, g0, total, n_ids);
+    ShortAhead ahead2 = short_ahead(a, g0 + gstride, total, n_ids);
+    ShortRow<E> row1 = short_row<E>(tabs, a, ahead1, g0, total, n_ids, eg);
     for (; (uint64_t)tile * bags_per_block < total; tile += gridDim.x) {
         const uint32_t g = tile * bags_per_block + lb;
         const bool live = g < total;
-        int32_t p = nx_p, p1 = nx_p1;
-        const int32_t spec_id = nx_id;
-        {   // the next tile's offsets and speculative ids
-            const uint64_t tn = (uint64_t)tile + gridDim.x;
-            const uint64_t gn = tn * bags_per_block + lb;
-            if (gn < total) {
-                nx_p = __ldg(a.offsets + gn);
-                nx_p1 = __ldg(a.offsets + gn + 1);
-                nx_id = (int64_t)gn < n_ids ? __ldg(a.indices + gn) : 0;
-            }
-        }
+        const ShortAhead cur = ahead1;
+        const ShortRow<E> crow = row1;
+        ahead1 = ahead2;
+        ahead2 = short_ahead(a, (uint64_t)g + 2 * gstride, total, n_ids);
+        row1 = short_row<E>(tabs, a, ahead1, (uint64_t)g + gstride, total, n_ids, eg);
+
         const int t = live ? (int)(g / batch) : 0;
         const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
+        int32_t p = cur.p, p1 = cur.p1;
         if (live)
             clamp_bag(p, p1, n_ids, eg == 0, a.flags);
         else
@@ -384,10 +418,12 @@ __device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const Bag
         for (int k = 0; k < E / 2; ++k)
             acc2[k] = make_float2(0.0f, 0.0f);
         bool bad = false;
-        if (p1 == p + 1) {  // one id: the speculative load holds it when it sits at position g
-            const uint32_t id = (uint32_t)(p == (int32_t)g ? spec_id : __ldg(a.indices + p));
+        if (crow.ready) {
+            accumulate_row<E>(crow.w, crow.sb, acc2);
+        } else if (p1 == p + 1) {
+            const uint32_t id = (uint32_t)__ldg(a.indices + p);
             if (id < tv.n_rows)
-                accumulate_row<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)),
+                accumulate_row<E>(__ldg(reinterpret_cast<const typename CodeVec<E>::T *>(tv.codes + (uint64_t)id * tv.ld)),
                                   __ldg(tv.sb + id), acc2);
             else
                 bad = true;
@@ -420,7 +456,7 @@ __device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const Bag
 }
 
 template <int E, int ISL>
-__global__ void __launch_bounds__(kBagThreads) embbag_kernel(const __grid_constant__ BagTables tabs,
+__global__ void __launch_bounds__(kBagThreads, E == 16 ? 4 : 1) embbag_kernel(const __grid_constant__ BagTables tabs,
                                                              const BagArgs a)
 {
     __shared__ __align__(16) float stage[(kBagThreads / 32) * 32 * (E + 4)];

@@ -21,9 +21,11 @@
 // quotient. The kernel instead forms u = sat(fma(x, r, -lo*r)) with r = rcp(w),
 // w = hi - lo (= 15 s up to one rounding), and rounds 15u with a magic-number add.
 // |15u - (x - lo)/s| <= 5.6e-6 + 9e-7 * |lo * r| (rcp error <= 1 ulp), so 15u rounds
-// like the IEEE quotient unless it lies within the margin 2^-16 + 2^-19 * |lo * r|
-// of a half-integer; such elements (a few in 10^5) are recomputed with IEEE
-// division. The codes the search sees are therefore exactly the IEEE ones.
+// like the IEEE quotient unless both lie within the margin m = 2^-16 + 2^-19 K of a
+// half-integer (K bounds |lo * r| over the row's walk). Then |e| / s is within
+// about m of 1/2 for either code, so an element whose e^2 falls in a narrow window
+// around s^2 / 4 (a few in 10^5) is recomputed with IEEE division. The codes the
+// search sees are therefore exactly the IEEE ones.
 //
 // s = w / 15 uses Markstein's correction step for a known divisor (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000 processor",
@@ -42,8 +44,8 @@ constexpr int kMoves = 168;              // moves while width > 0.16 * range
 constexpr float kLevels = 15.0f;         // 2^4 - 1
 constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23: x + kMagic rounds x in [0, 2^22) to an integer
 constexpr float kInv15 = 1.0f / 15.0f;   // RN(1/15)
-constexpr float kGap0 = 0.5f - 1.52587890625e-05f;  // 0.5 - 2^-16
-constexpr float kGapLo = 1.9073486328125e-06f;     // 2^-19 per unit of |lo * r|
+constexpr float kGap1 = 1.52587890625e-05f;    // tie margin on 15u: 2^-16 ...
+constexpr float kGapLo = 1.9073486328125e-06f;  // ... plus 2^-19 per unit of |lo * r|
 constexpr float kFastWMin = 1.0e-36f;    // w in [kFastWMin, kFastWMax]: s normal, 1/w normal
 constexpr float kFastWMax = 1.0e36f;
 constexpr float kFastLoR = 65536.0f;     // |lo * r| above this: IEEE path
@@ -100,13 +102,31 @@ __device__ __forceinline__ void row_minmax(float &mn, float &mx)
 
 // One clip range [lo, hi] of the search, with what its elements share.
 struct Clip {
-    float lo, s;      // bias and scale of the candidate quantizer
-    float r, nlr;     // rcp(hi - lo) and -RN(lo * r): u = sat(fma(x, r, nlr))
-    float thr;        // |15u - q| above thr: too close to a rounding tie, recompute
-    uint32_t c_lo, c_span;  // e^2 with bits in [c_lo, c_lo + c_span): near a tie
+    float lo, s;            // bias and scale of the candidate quantizer
+    float r, nlr;           // rcp(hi - lo) and -RN(lo * r): u = sat(fma(x, r, nlr))
+    uint32_t c_lo, c_span;  // e^2 with bits in [c_lo, c_lo + c_span): near a rounding tie
 };
 
-__device__ __forceinline__ Clip clip_fast(float lo, float hi, float thr)
+// The tie window of a row, as multiples of s^2. Where the division-free code can
+// differ from the IEEE one, 15u and the exact quotient lie within the margin m of
+// a half-integer, so |e| / s = |quotient - q| is within b of 1/2 for either code,
+// b = m plus the rounding of xhat and e (below 2^-24 (15 K + 16)); 2 m + 2^-16
+// covers both. The window is [(1/2 - b)^2, (1/2 + b)^2], widened by 1e-6 for the
+// rounding of s^2 and of the bounds.
+struct TieWindow {
+    float kl, kh;
+};
+
+__device__ __forceinline__ TieWindow tie_window(float margin)
+{
+    const float b = __fmaf_rn(2.0f, margin, 1.52587890625e-05f);
+    TieWindow t;
+    t.kl = __fmul_rn(__fmaf_rn(-b, 1.0f - b, 0.25f), 0.999999f);
+    t.kh = __fmul_rn(__fmaf_rn(b, 1.0f + b, 0.25f), 1.000001f);
+    return t;
+}
+
+__device__ __forceinline__ Clip clip_fast(float lo, float hi, const TieWindow &tw)
 {
     Clip c;
     c.lo = lo;
@@ -114,15 +134,9 @@ __device__ __forceinline__ Clip clip_fast(float lo, float hi, float thr)
     c.r = rcp_approx(w);
     c.nlr = __fmul_rn(-lo, c.r);
     c.s = div15(w);
-    c.thr = thr;
-    // |e| / s within b of 1/2 where b = 0.5 - thr (the tie margin) widened for the
-    // rounding of xhat and e: e^2 in s^2 [(1/2 - b')^2, (1/2 + b')^2]
-    const float b = __fmaf_rn(2.0f, 0.5f - thr, 1.52587890625e-05f);
     const float s2 = __fmul_rn(c.s, c.s);
-    const float lo_c = __fmul_rn(s2, __fmaf_rn(-b, 1.0f - b, 0.25f) * 0.999999f);
-    const float hi_c = __fmul_rn(s2, __fmaf_rn(b, 1.0f + b, 0.25f) * 1.000001f);
-    c.c_lo = __float_as_uint(lo_c);
-    c.c_span = __float_as_uint(hi_c) - c.c_lo;
+    c.c_lo = __float_as_uint(__fmul_rn(s2, tw.kl));
+    c.c_span = __float_as_uint(__fmul_rn(s2, tw.kh)) - c.c_lo;
     return c;
 }
 
@@ -164,14 +178,6 @@ __device__ __forceinline__ void errors_packed(const float2 (&xp)[H], const Clip 
         if (!valid_y<H, HAS_Y, FULL>(kbase, h, d))
             C[h].y = 0.0f;
     }
-}
-
-// The tie distance 15u - q of one element, by the same operations as errors_packed.
-__device__ __forceinline__ float tie_distance(float x, const Clip &c)
-{
-    const float u = fma_sat(x, c.r, c.nlr);
-    const float nq = __fmaf_rn(__fmaf_rn(u, kLevels, kMagic), -1.0f, kMagic);
-    return __fmaf_rn(u, kLevels, nq);
 }
 
 // Recomputes with IEEE division every element whose fast code was too close to a tie.
@@ -219,7 +225,8 @@ __device__ __forceinline__ float tree_sum2(float2 (&C)[H])
 // otherwise IEEE division for every element. All lanes of a row see the same losses.
 template <int H, bool HAS_Y, bool FULL, bool FAST, int W>
 __device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, int d, float mn, float mx,
-                                            float step, float thr, float &lbest, float &fbi, float &fbj)
+                                            float step, const TieWindow &tw, float &lbest, float &fbi,
+                                            float &fbj)
 {
     float fi = 0.0f, fj = 0.0f;  // grid indices as exact small floats (i + j <= 168)
     float lo_i = __fmaf_rn(0.0f, step, mn), hi_j = __fmaf_rn(-0.0f, step, mx);
@@ -228,7 +235,7 @@ __device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, in
         // left candidate (i+1, j) = a, right candidate (i, j+1) = b
         float2 Ca[H], Cb[H];
         if constexpr (FAST) {
-            const Clip ca = clip_fast(lo_i1, hi_j, thr), cb = clip_fast(lo_i, hi_j1, thr);
+            const Clip ca = clip_fast(lo_i1, hi_j, tw), cb = clip_fast(lo_i, hi_j1, tw);
             // each candidate is reduced as soon as its errors exist; a candidate with
             // an element too close to a rounding tie (rare) is evaluated again with
             // the IEEE fix-up
@@ -348,11 +355,11 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
         const float w_min = __fmul_rn(step, 30.0f);
         const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
         const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
-        const float thr = __fmaf_rn(K, -kGapLo, kGap0);
+        const TieWindow tw = tie_window(__fmaf_rn(K, kGapLo, kGap1));
         if (fast)
-            greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, thr, lbest, fbi, fbj);
+            greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
         else
-            greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, thr, lbest, fbi, fbj);
+            greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
     }
     const int bi = (int)fbi, bj = (int)fbj;
 
