@@ -21,10 +21,10 @@
 // quotient. The kernel instead forms u = sat(fma(x, r, -lo*r)) with r = rcp(w),
 // w = hi - lo (= 15 s up to one rounding), and rounds 15u with a magic-number add.
 // |15u - (x - lo)/s| <= 5.6e-6 + 9e-7 * |lo * r| (rcp error <= 1 ulp), so 15u rounds
-// like the IEEE quotient unless both lie within the margin m = 2^-16 + 2^-19 K of a
-// half-integer (K bounds |lo * r| over the row's walk). Then |e| / s is within
-// about m of 1/2 for either code, so an element whose e^2 falls in a narrow window
-// around s^2 / 4 (a few in 10^5) is recomputed with IEEE division. The codes the
+// like the IEEE quotient unless both lie within about 6e-6 + 9e-7 K of a
+// half-integer (K bounds |lo * r| over the row's walk). Then |e| / s is within about
+// that of 1/2 for either code, so an element whose e^2 falls in a narrow window
+// around s^2 / 4 (about 3 in 10^5) is recomputed with IEEE division. The codes the
 // search sees are therefore exactly the IEEE ones.
 //
 // s = w / 15 uses Markstein's correction step for a known divisor (P. Markstein,
@@ -44,8 +44,6 @@ constexpr int kMoves = 168;              // moves while width > 0.16 * range
 constexpr float kLevels = 15.0f;         // 2^4 - 1
 constexpr float kMagic = 12582912.0f;    // 1.5 * 2^23: x + kMagic rounds x in [0, 2^22) to an integer
 constexpr float kInv15 = 1.0f / 15.0f;   // RN(1/15)
-constexpr float kGap1 = 1.52587890625e-05f;    // tie margin on 15u: 2^-16 ...
-constexpr float kGapLo = 1.9073486328125e-06f;  // ... plus 2^-19 per unit of |lo * r|
 constexpr float kFastWMin = 1.0e-36f;    // w in [kFastWMin, kFastWMax]: s normal, 1/w normal
 constexpr float kFastWMax = 1.0e36f;
 constexpr float kFastLoR = 65536.0f;     // |lo * r| above this: IEEE path
@@ -107,19 +105,21 @@ struct Clip {
     uint32_t c_lo, c_span;  // e^2 with bits in [c_lo, c_lo + c_span): near a rounding tie
 };
 
-// The tie window of a row, as multiples of s^2. Where the division-free code can
-// differ from the IEEE one, 15u and the exact quotient lie within the margin m of
-// a half-integer, so |e| / s = |quotient - q| is within b of 1/2 for either code,
-// b = m plus the rounding of xhat and e (below 2^-24 (15 K + 16)); 2 m + 2^-16
-// covers both. The window is [(1/2 - b)^2, (1/2 + b)^2], widened by 1e-6 for the
-// rounding of s^2 and of the bounds.
+// The tie window of a row, as multiples of s^2. With q the division-free code and
+// y = (x - lo) / s exactly: |15u - y| <= 3.7e-6 + 8.9e-7 K (the rounding of r, -lo*r,
+// u and s; K bounds |lo * r| over the row's walk) and the IEEE quotient is within
+// 1.9e-6 of y, so where the two codes differ, |y - q| is within 5.6e-6 + 8.9e-7 K of
+// 1/2, and the computed |e| / s within b_min = 6.6e-6 + 1.8e-6 K of 1/2 (the rounding
+// of xhat and e adds at most 2^-24 (15 K + 16)). The window uses b = 1.2e-5 + 3e-6 K,
+// about 1.7 b_min: e^2 in s^2 [(1/2 - b)^2, (1/2 + b)^2], widened by 1e-6 for the
+// rounding of s^2, of the bounds and of e^2.
 struct TieWindow {
     float kl, kh;
 };
 
-__device__ __forceinline__ TieWindow tie_window(float margin)
+__device__ __forceinline__ TieWindow tie_window(float K)
 {
-    const float b = __fmaf_rn(2.0f, margin, 1.52587890625e-05f);
+    const float b = __fmaf_rn(K, 3.0e-6f, 1.2e-5f);
     TieWindow t;
     t.kl = __fmul_rn(__fmaf_rn(-b, 1.0f - b, 0.25f), 0.999999f);
     t.kh = __fmul_rn(__fmaf_rn(b, 1.0f + b, 0.25f), 1.000001f);
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
         const float w_min = __fmul_rn(step, 30.0f);
         const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
         const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
-        const TieWindow tw = tie_window(__fmaf_rn(K, kGapLo, kGap1));
+        const TieWindow tw = tie_window(K);
         if (fast)
             greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
         else

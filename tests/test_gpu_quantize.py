@@ -112,3 +112,32 @@ def test_zero_rows_and_repeat_calls(cuda_device):
     import torch
     dq.dq_quantize_rows_int4(None, 0, 16, 16, None, 8, None)
     torch.cuda.synchronize()
+
+
+def _tie_rows(n, d, seed):
+    """Rows whose elements sit at (or within an ulp of) half-integer quotients for
+    both candidates of the first greedy move, so the division-free codes have to
+    defer to IEEE division on most elements."""
+    r = np.random.default_rng(seed)
+    rows = []
+    for _ in range(n):
+        R = np.float32(r.uniform(0.5, 4.0))
+        off = np.float32(r.uniform(-2, 2))
+        step = np.float32(R / np.float32(200))
+        lo1 = np.float32(off + step)             # left candidate: (xmin + step, xmax)
+        hi1 = np.float32(off + R - step)         # right candidate: (xmin, xmax - step)
+        s_l = np.float32(np.float32((off + R) - lo1) / np.float32(15))
+        s_r = np.float32(np.float32(hi1 - off) / np.float32(15))
+        k = r.integers(0, 15, d - 2)
+        half = np.where(r.random(d - 2) < 0.5, lo1 + (k + 0.5) * s_l, off + (k + 0.5) * s_r).astype(np.float32)
+        # each tie value itself or its neighbour one ulp up or down
+        direction = np.where(r.random(d - 2) < 0.5, np.inf, -np.inf).astype(np.float32)
+        half = np.where(r.random(d - 2) < 0.5, half, np.nextafter(half, direction))
+        rows.append(np.concatenate([[off, off + R], half]).astype(np.float32))
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("d", [16, 64])
+def test_rows_built_on_rounding_ties(cuda_device, d):
+    x = _tie_rows(800 if d == 16 else 200, d, d)
+    assert_quant_parity(x)
