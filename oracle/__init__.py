@@ -62,6 +62,8 @@ def lib():
             L.oracle_quantize_rows.restype = i32
             L.oracle_dequantize_rows.argtypes = [vp, i64, vp, i64, i32, vp, i64]
             L.oracle_dequantize_rows.restype = i32
+            L.oracle_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp]
+            L.oracle_row_l2_error.restype = ctypes.c_double
             L.oracle_embbag.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, i32]
             L.oracle_embbag.restype = i64
             _lib = L
@@ -141,6 +143,19 @@ def dequantize_rows(codes: np.ndarray, scale_bias: np.ndarray, d: int) -> np.nda
     if rc != 0:
         raise ValueError("oracle_dequantize_rows: bad arguments")
     return out
+
+
+def row_l2_error(x: np.ndarray, codes: np.ndarray, scale_bias: np.ndarray):
+    """(per-row normalized l2 error float64 [n], their sum float64)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sb = np.ascontiguousarray(scale_bias, dtype=np.uint16)
+    n, d = x.shape
+    err = np.zeros(n, np.float64)
+    tot = lib().oracle_row_l2_error(_p(x), n, d, d, _p(codes), codes.shape[1], _p(sb), _p(err))
+    if np.isnan(tot):
+        raise ValueError("oracle_row_l2_error: bad arguments")
+    return err, float(tot)
 
 
 def embbag(tables, d: int, indices: np.ndarray, offsets: np.ndarray, batch: int,

@@ -40,6 +40,11 @@
  *      nibble 0. The plain min/max quantizer is step 5 skipped.
  *
  *   Dequantize: xhat_k = fma(q_k, S, B).
+ *   Normalized l2 error of a row (the quality measure of "Post-Training 4-bit
+ *   Quantization on Embedding Tables", 提出的方法 bullet 5; the pages do not define it,
+ *   the reading taken is): sqrt(sum_k (x_k - xhat_k)^2) / sqrt(sum_k x_k^2), both sums
+ *   in binary64 over the binary64 values of the binary32 x and xhat, in index order;
+ *   a row with sum x^2 = 0 has error 0 if it is reconstructed exactly, else +inf.
  *   Embedding bag: out[b][t*d + k] = sum over the bag's ids p of xhat_{p,k}, summed
  *   in binary64 in index order and rounded once to binary32; an empty bag gives +0.
  *
@@ -382,6 +387,33 @@ int32_t oracle_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uin
         }
     }
     return 0;
+}
+
+/* Normalized l2 error of each of n rows (binary64); returns the sum over rows
+ * (binary64, index order), or NAN on bad arguments. row_err may be NULL. */
+double oracle_row_l2_error(const float *x, int64_t n, int32_t d, int64_t x_ld, const uint8_t *codes,
+                           int64_t codes_ld, const uint16_t *scale_bias, double *row_err)
+{
+    if (n < 0 || d < 1 || d > ORACLE_MAX_D || x_ld < d || codes_ld < (d + 1) / 2)
+        return NAN;
+    double total = 0.0;
+    for (int64_t row = 0; row < n; row++) {
+        float S = oracle_f16_to_f32(scale_bias[2 * row]);
+        float B = oracle_f16_to_f32(scale_bias[2 * row + 1]);
+        double se = 0.0, sx = 0.0;
+        for (int k = 0; k < d; k++) {
+            int q = (codes[row * codes_ld + k / 2] >> (4 * (k % 2))) & 0xf;
+            double xk = (double)x[row * x_ld + k];
+            double e = xk - (double)fmaf((float)q, S, B);
+            se += e * e;
+            sx += xk * xk;
+        }
+        double err = sx > 0.0 ? sqrt(se / sx) : (se > 0.0 ? INFINITY : 0.0);
+        if (row_err)
+            row_err[row] = err;
+        total += err;
+    }
+    return total;
 }
 
 typedef struct {
