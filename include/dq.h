@@ -147,6 +147,24 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
                              const int32_t *indices, const int32_t *offsets, int32_t batch,
                              float *out, uint32_t *d_flags, void *cuda_stream);
 
+/*
+ * dq_row_l2_error -- normalized l2 error of packed rows against their binary32
+ * originals: row_err[r] = sqrt(sum_k (x[r][k] - xhat_k)^2) / sqrt(sum_k x[r][k]^2),
+ * xhat_k = fma(q_k, scale, bias), both sums in binary64 (a row with sum x^2 = 0 gives
+ * 0 if reconstructed exactly, else +inf). ("Post-Training 4-bit Quantization on
+ * Embedding Tables", 提出的方法 / proposed method, bullet 5: quantization error as
+ * normalized l2 loss; 主要发现 / main findings, bullet 2.)
+ *
+ *   x, n_rows, d, x_ld            the binary32 rows, as for dq_quantize_rows_int4
+ *   codes, codes_ld, scale_bias   their packed form (scale_bias 4-byte aligned)
+ *   row_err     [n_rows] binary64 (output, nullable)
+ *   err_sum     device binary64 scalar (nullable): the sum of the row errors is ADDED
+ *               to it (atomically, in no fixed order); zero it before the call
+ */
+dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_ld,
+                          const uint8_t *codes, int64_t codes_ld, const uint16_t *scale_bias,
+                          double *row_err, double *err_sum, void *cuda_stream);
+
 /* Static text for a status code. */
 const char *dq_status_string(dq_status s);
 

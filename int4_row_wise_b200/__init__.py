@@ -8,10 +8,10 @@ libdq's kernels; there is no CPU path. If libdq.so is missing, the first call
 raises DqError (build it with `python -m int4_row_wise_b200.build`).
 
 Low-level calls with the C names:
-    dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd,
+    dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd, dq_row_l2_error,
     dq_status_string, dq_last_error, dq_version
 Convenience wrappers that allocate their outputs with torch:
-    quantize_rows, dequantize_rows, embbag
+    quantize_rows, dequantize_rows, embbag, row_l2_error
 """
 from __future__ import annotations
 
@@ -25,9 +25,9 @@ __all__ = [
     "DQ_MODE_GREEDY", "DQ_MODE_MINMAX",
     "DQ_FLAG_BAD_INDEX", "DQ_FLAG_BAD_OFFSETS", "DQ_FLAG_NONFINITE", "DQ_FLAG_FP16_OVERFLOW",
     "DQ_MAX_D", "DQ_MAX_TABLES", "DqError", "PackedTable", "lib_path", "load",
-    "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd",
+    "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_row_l2_error",
     "dq_status_string", "dq_last_error", "dq_version",
-    "quantize_rows", "dequantize_rows", "embbag",
+    "quantize_rows", "dequantize_rows", "embbag", "row_l2_error",
 ]
 
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA = 0, 1, 2, 3
@@ -73,6 +73,8 @@ def load():
             L.dq_dequantize_rows.restype = ctypes.c_int
             L.dq_embbag_int4_fwd.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp]
             L.dq_embbag_int4_fwd.restype = ctypes.c_int
+            L.dq_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp]
+            L.dq_row_l2_error.restype = ctypes.c_int
             L.dq_status_string.argtypes, L.dq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
             L.dq_last_error.argtypes, L.dq_last_error.restype = [], ctypes.c_char_p
             L.dq_version.argtypes, L.dq_version.restype = [], i32
@@ -133,6 +135,14 @@ def dq_dequantize_rows(codes, codes_ld: int, scale_bias, n_rows: int, d: int, ou
     st = load().dq_dequantize_rows(_ptr(codes), codes_ld, _ptr(scale_bias), n_rows, d, _ptr(out), out_ld,
                                    _stream(stream))
     _check(st, "dq_dequantize_rows")
+
+
+def dq_row_l2_error(x, n_rows: int, d: int, x_ld: int, codes, codes_ld: int, scale_bias, row_err=None,
+                    err_sum=None, stream=None) -> None:
+    """C: dq_row_l2_error (err_sum is accumulated into)."""
+    st = load().dq_row_l2_error(_ptr(x), n_rows, d, x_ld, _ptr(codes), codes_ld, _ptr(scale_bias),
+                                _ptr(row_err), _ptr(err_sum), _stream(stream))
+    _check(st, "dq_row_l2_error")
 
 
 class PackedTable(NamedTuple):
@@ -202,3 +212,14 @@ def embbag(tables: Sequence, d: int, indices, offsets, batch: int, d_flags=None,
     out = torch.empty((batch, len(tables) * d), dtype=torch.float32, device=indices.device)
     dq_embbag_int4_fwd(tables, d, indices, offsets, batch, out, d_flags, stream)
     return out
+
+
+def row_l2_error(x, codes, scale_bias, stream=None):
+    """Normalized l2 error of each row of x against its packed form: (float64 [n], mean)."""
+    import torch
+    n, d = x.shape
+    err = torch.empty(n, dtype=torch.float64, device=x.device)
+    tot = torch.zeros(1, dtype=torch.float64, device=x.device)
+    dq_row_l2_error(x, n, d, x.stride(0) if n > 1 else d, codes, codes.stride(0) if n > 1 else codes.shape[1],
+                    scale_bias, err, tot, stream)
+    return err, tot / max(n, 1)

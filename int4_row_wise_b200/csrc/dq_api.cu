@@ -176,6 +176,34 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
     return launched(dq::launch_embbag(tabs, a, sms, (cudaStream_t)cuda_stream), "embbag");
 }
 
+dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, const uint8_t *codes,
+                          int64_t codes_ld, const uint16_t *scale_bias, double *row_err, double *err_sum,
+                          void *cuda_stream)
+{
+    if (n_rows < 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (x_ld < d)
+        return fail(DQ_ERR_INVALID_ARG, "x_ld = %lld < d = %d", (long long)x_ld, d);
+    if (codes_ld < (d + 1) / 2)
+        return fail(DQ_ERR_INVALID_ARG, "codes_ld = %lld < (d+1)/2 = %d", (long long)codes_ld, (d + 1) / 2);
+    if (n_rows > 0 && (!x || !codes || !scale_bias))
+        return fail(DQ_ERR_INVALID_ARG, "x, codes and scale_bias must be non-NULL when n_rows > 0");
+    if (n_rows > 0 && (reinterpret_cast<uintptr_t>(scale_bias) & 3) != 0)
+        return fail(DQ_ERR_INVALID_ARG, "scale_bias must be 4-byte aligned");
+    if (n_rows == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::L2Args a{x, n_rows, x_ld, d, codes, codes_ld, scale_bias, row_err, err_sum};
+    return launched(dq::launch_row_l2(a, sms, (cudaStream_t)cuda_stream), "row_l2_error");
+}
+
 const char *dq_status_string(dq_status s)
 {
     switch (s) {

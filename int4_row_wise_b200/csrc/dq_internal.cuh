@@ -41,6 +41,17 @@ struct BagTables {
     int64_t codes_ld[DQ_MAX_TABLES];
 };
 
+struct L2Args {
+    const float *x;
+    int64_t n, ld;
+    int d;
+    const uint8_t *codes;
+    int64_t codes_ld;
+    const uint16_t *scale_bias;
+    double *row_err;
+    double *err_sum;
+};
+
 struct BagArgs {
     int T, d, batch;
     const int32_t *indices;
@@ -52,6 +63,7 @@ struct BagArgs {
 cudaError_t launch_quantize(const QuantArgs &a, int mode, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream);
 
 __device__ __forceinline__ void raise_flag(uint32_t *flags, uint32_t bit)
 {
