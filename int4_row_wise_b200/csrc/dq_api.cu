@@ -172,7 +172,7 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
         return st;
     if (fault_injected())
         return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
-    dq::BagArgs a{n_tables, d, batch, indices, offsets, out, d_flags};
+    dq::BagArgs a{n_tables, d, batch, indices, offsets, out, d_flags, dq::make_batch_div((uint32_t)batch)};
     return launched(dq::launch_embbag(tabs, a, sms, (cudaStream_t)cuda_stream), "embbag");
 }
 

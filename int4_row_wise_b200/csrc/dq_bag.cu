@@ -290,7 +290,7 @@ __device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagA
     for (uint32_t tile = blockIdx.x; (uint64_t)tile * bags_per_block < total; tile += gridDim.x) {
         const uint32_t g = tile * bags_per_block + lb;
         const bool live = g < total;
-        const int t = live ? (int)(g / batch) : 0;
+        const int t = live ? (int)div_batch(g, a.div) : 0;
         const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
         int32_t p = 0, p1 = 0;
         if (live) {
@@ -362,7 +362,7 @@ __device__ __forceinline__ ShortRow<E> short_row(const BagTables &tabs, const Ba
     ShortRow<E> r;
     r.ready = false;
     if (g < total && (int64_t)s.p == (int64_t)g && s.p1 == s.p + 1 && s.p1 <= n_ids) {
-        const int t = (int)((uint32_t)g / (uint32_t)a.batch);
+        const int t = (int)div_batch((uint32_t)g, a.div);
         const TableView tv = table_view(tabs, t, eg, E);
         if ((uint32_t)s.id < tv.n_rows) {
             r.w = __ldg(reinterpret_cast<const typename CodeVec<E>::T *>(tv.codes + (uint64_t)(uint32_t)s.id * tv.ld));
@@ -405,7 +405,7 @@ __device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const Bag
         ahead2 = short_ahead(a, (uint64_t)g + 2 * gstride, total, n_ids);
         row1 = short_row<E>(tabs, a, ahead1, (uint64_t)g + gstride, total, n_ids, eg);
 
-        const int t = live ? (int)(g / batch) : 0;
+        const int t = live ? (int)div_batch(g, a.div) : 0;
         const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
         int32_t p = cur.p, p1 = cur.p1;
         if (live)

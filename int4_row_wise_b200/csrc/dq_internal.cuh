@@ -52,13 +52,39 @@ struct L2Args {
     double *err_sum;
 };
 
+// Division of 32-bit unsigned n by the invariant batch (T. Granlund, P. Montgomery,
+// "Division by invariant integers using multiplication", PLDI 1994, Fig. 4.1):
+// t = umulhi(m, n), n / batch = (t + ((n - t) >> sh1)) >> sh2.
+struct BatchDiv {
+    uint32_t m, sh1, sh2;
+};
+
 struct BagArgs {
     int T, d, batch;
     const int32_t *indices;
     const int32_t *offsets;
     float *out;
     uint32_t *flags;
+    BatchDiv div;
 };
+
+inline BatchDiv make_batch_div(uint32_t dvs)
+{
+    uint32_t l = 0;
+    while ((1ull << l) < dvs)
+        ++l;
+    BatchDiv r;
+    r.m = (uint32_t)(((1ull << 32) * ((1ull << l) - dvs)) / dvs + 1);
+    r.sh1 = l < 1 ? l : 1;
+    r.sh2 = l > 1 ? l - 1 : 0;
+    return r;
+}
+
+__device__ __forceinline__ uint32_t div_batch(uint32_t n, const BatchDiv &v)
+{
+    const uint32_t t = __umulhi(v.m, n);
+    return (t + ((n - t) >> v.sh1)) >> v.sh2;
+}
 
 cudaError_t launch_quantize(const QuantArgs &a, int mode, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t stream);
