@@ -64,6 +64,9 @@ def lib():
             L.oracle_dequantize_rows.restype = i32
             L.oracle_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp]
             L.oracle_row_l2_error.restype = ctypes.c_double
+            L.oracle_embbag_bwd_sgd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i64, vp,
+                                                ctypes.c_float, i32]
+            L.oracle_embbag_bwd_sgd.restype = i64
             L.oracle_embbag.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, i32]
             L.oracle_embbag.restype = i64
             _lib = L
@@ -180,3 +183,35 @@ def embbag(tables, d: int, indices: np.ndarray, offsets: np.ndarray, batch: int,
     if skipped < 0:
         raise ValueError("oracle_embbag: bad arguments")
     return out, mag, int(skipped)
+
+
+BWD_WINDOW = 64
+BAD_OFFSETS = -2
+
+
+def embbag_bwd_sgd(masters, codes, scale_bias, d: int, indices: np.ndarray, offsets: np.ndarray,
+                   batch: int, grad: np.ndarray, lr: float, mode: int = GREEDY) -> int:
+    """Bag backward, SGD step on the binary32 masters and re-quantization of the touched
+    rows, all in place. masters: list of float32 [n, ld]; codes: list of uint8 [n, cld];
+    scale_bias: list of uint16 [n, 2]; grad: float32 [batch, T*d]. Returns the number of
+    invalid ids, or BAD_OFFSETS when the offsets are not a CSR array (nothing changed)."""
+    T = len(masters)
+    for w, c, sb in zip(masters, codes, scale_bias):
+        assert w.dtype == np.float32 and w.flags["C_CONTIGUOUS"]
+        assert c.dtype == np.uint8 and c.flags["C_CONTIGUOUS"] and c.shape[0] == w.shape[0]
+        assert sb.dtype == np.uint16 and sb.flags["C_CONTIGUOUS"] and sb.shape == (w.shape[0], 2)
+
+    def ptrs(arrs):
+        return ctypes.cast((ctypes.c_void_p * T)(*[a.ctypes.data for a in arrs]), ctypes.c_void_p)
+
+    wld = np.array([w.shape[1] for w in masters], np.int64)
+    cld = np.array([c.shape[1] for c in codes], np.int64)
+    nrows = np.array([w.shape[0] for w in masters], np.int64)
+    idx = np.ascontiguousarray(indices, dtype=np.int32)
+    off = np.ascontiguousarray(offsets, dtype=np.int32)
+    g = np.ascontiguousarray(grad, dtype=np.float32)
+    r = lib().oracle_embbag_bwd_sgd(ptrs(masters), _p(wld), ptrs(codes), _p(cld), ptrs(scale_bias), _p(nrows),
+                                    T, d, _p(idx), _p(off), batch, int(idx.size), _p(g), np.float32(lr), mode)
+    if r == -1:
+        raise ValueError("oracle_embbag_bwd_sgd: bad arguments")
+    return int(r)

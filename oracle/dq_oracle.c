@@ -47,7 +47,25 @@
  *   a row with sum x^2 = 0 has error 0 if it is reconstructed exactly, else +inf.
  *   Embedding bag: out[b][t*d + k] = sum over the bag's ids p of xhat_{p,k}, summed
  *   in binary64 in index order and rounded once to binary32; an empty bag gives +0.
- *
+ *   Bag backward, SGD step and re-quantization of the touched rows (the training
+ *   step of the DQRM repository page: embeddings trained at INT4 with quantization-
+ *   aware training on binary32 masters; the pages fix no arithmetic for it, the
+ *   reading taken is):
+ *   a. Offsets must be a CSR array: offsets[0] = 0, nondecreasing, offsets[T*B] =
+ *      the number of indices; otherwise nothing changes. Every position p of bag
+ *      (t, b) with a valid id gives an entry (key = row_base[t] + id, p), row_base[t]
+ *      = rows of the tables before t. Invalid ids give no entry.
+ *   b. The entries are sorted by (key, p). Their list is cut into windows of 64
+ *      consecutive entries (positions 0..63, 64..127, ...).
+ *   c. Gradient of a row, element k: the binary64 sum, from +0 in list order, of
+ *      g[b][t*d + k] over the row's entries inside each window; these window parts
+ *      are added, from +0 in window order, in binary64; G_k is that total rounded
+ *      once to binary32.
+ *   d. W[id][k] = fma(-lr, G_k, W[id][k]) (binary32, rounded once).
+ *   e. Each touched row (one with at least one entry) is quantized again from its new
+ *      master values by the quantizer above (greedy or min/max); other rows keep
+ *      their codes.
+ * *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared -pthread
  * (no FMA contraction and no excess precision, so every C operator below is one
  * IEEE binary32 operation; fmaf() is the C library's correctly rounded FMA).
@@ -474,6 +492,111 @@ static void *bag_worker(void *arg)
         }
     }
     return NULL;
+}
+
+#define ORACLE_BWD_WINDOW 64
+
+typedef struct {
+    uint32_t key;
+    int32_t bag;
+    int64_t pos;
+} bwd_entry;
+
+static int entry_cmp(const void *pa, const void *pb)
+{
+    const bwd_entry *a = (const bwd_entry *)pa, *b = (const bwd_entry *)pb;
+    if (a->key != b->key)
+        return a->key < b->key ? -1 : 1;
+    return a->pos < b->pos ? -1 : (a->pos > b->pos ? 1 : 0);
+}
+
+/* Steps a-e of the bag backward on T tables sharing d: masters W[t] (row stride
+ * w_ld[t]) and packed tables codes[t]/scale_bias[t] (code row stride codes_ld[t]),
+ * n_rows[t] rows each; grad is [B][T*d]. Returns the number of invalid ids, -2 if the
+ * offsets are not a CSR array (nothing changed), -1 on bad arguments. */
+int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *const *codes,
+                              const int64_t *codes_ld, uint16_t *const *scale_bias,
+                              const int64_t *n_rows, int32_t T, int32_t d, const int32_t *indices,
+                              const int32_t *offsets, int32_t B, int64_t n_indices, const float *grad,
+                              float lr, int32_t mode)
+{
+    if (T < 1 || d < 1 || d > ORACLE_MAX_D || B < 0 || n_indices < 0)
+        return -1;
+    int64_t G = (int64_t)T * B;
+    if (offsets[0] != 0 || offsets[G] != n_indices)
+        return -2;
+    for (int64_t g = 0; g < G; g++)
+        if (offsets[g + 1] < offsets[g])
+            return -2;
+    /* a. entries */
+    int64_t *row_base = (int64_t *)malloc(sizeof(int64_t) * (size_t)T);
+    int64_t total = 0;
+    for (int t = 0; t < T; t++) {
+        row_base[t] = total;
+        total += n_rows[t];
+    }
+    bwd_entry *e = (bwd_entry *)malloc(sizeof(bwd_entry) * (size_t)(n_indices > 0 ? n_indices : 1));
+    int64_t ne = 0, invalid = 0;
+    for (int64_t g = 0; g < G; g++) {
+        int t = (int)(g / (B > 0 ? B : 1));
+        for (int64_t p = offsets[g]; p < offsets[g + 1]; p++) {
+            int32_t id = indices[p];
+            if (id < 0 || (int64_t)id >= n_rows[t]) {
+                invalid++;
+                continue;
+            }
+            e[ne].key = (uint32_t)(row_base[t] + id);
+            e[ne].bag = (int32_t)g;
+            e[ne].pos = p;
+            ne++;
+        }
+    }
+    /* b. sort by (key, p) */
+    qsort(e, (size_t)ne, sizeof(bwd_entry), entry_cmp);
+    double *part = (double *)malloc(sizeof(double) * (size_t)d);
+    double *sum = (double *)malloc(sizeof(double) * (size_t)d);
+    float cbuf[ORACLE_MAX_D];
+    for (int64_t s0 = 0; s0 < ne;) {
+        int64_t s1 = s0;
+        while (s1 < ne && e[s1].key == e[s0].key)
+            s1++;
+        int t = 0;
+        while (t + 1 < T && (int64_t)e[s0].key >= row_base[t + 1])
+            t++;
+        int64_t id = (int64_t)e[s0].key - row_base[t];
+        /* c. window parts, then their sum */
+        for (int k = 0; k < d; k++)
+            sum[k] = 0.0;
+        for (int64_t w0 = s0; w0 < s1;) {
+            int64_t w1 = (w0 / ORACLE_BWD_WINDOW + 1) * ORACLE_BWD_WINDOW;
+            if (w1 > s1)
+                w1 = s1;
+            for (int k = 0; k < d; k++)
+                part[k] = 0.0;
+            for (int64_t i = w0; i < w1; i++) {
+                int64_t b = e[i].bag - (int64_t)t * B;
+                const float *gr = grad + b * (int64_t)T * d + (int64_t)t * d;
+                for (int k = 0; k < d; k++)
+                    part[k] = part[k] + (double)gr[k];
+            }
+            for (int k = 0; k < d; k++)
+                sum[k] = sum[k] + part[k];
+            w0 = w1;
+        }
+        /* d. SGD step */
+        float *w = W[t] + id * w_ld[t];
+        for (int k = 0; k < d; k++)
+            w[k] = fmaf(-lr, (float)sum[k], w[k]);
+        /* e. re-quantize the row */
+        search_result r = search_row(w, d, mode, cbuf, NULL, NULL, NULL, NULL, NULL);
+        finish_row(w, d, &r, codes[t] + id * codes_ld[t], scale_bias[t] + 2 * id);
+        s0 = s1;
+    }
+    free(part);
+    free(sum);
+    free(e);
+    free(row_base);
+    return invalid;
 }
 
 /* Sum-pooled lookup over T packed tables sharing d. indices/offsets as the CUDA
