@@ -48,6 +48,7 @@
 #ifndef DQ_H
 #define DQ_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -164,6 +165,65 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
 dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_ld,
                           const uint8_t *codes, int64_t codes_ld, const uint16_t *scale_bias,
                           double *row_err, double *err_sum, void *cuda_stream);
+
+/* One table of the bag backward: its binary32 master rows and their packed form.
+ * All pointers are device pointers. */
+typedef struct dq_master_table {
+    float *master;          /* [n_rows][master_ld] binary32, 4-byte aligned; touched rows updated */
+    int64_t master_ld;      /* >= d */
+    uint8_t *codes;         /* packed rows (format above); touched rows rewritten */
+    int64_t codes_ld;       /* >= (d+1)/2 */
+    uint16_t *scale_bias;   /* [n_rows][2] binary16 patterns, 2-byte aligned; touched rows rewritten */
+    int64_t n_rows;         /* >= 0; all tables together hold at most 2^32 - 2 rows */
+} dq_master_table;
+
+/*
+ * dq_embbag_int4_bwd_workspace_bytes -- device workspace that dq_embbag_int4_bwd_sgd
+ * needs for n_indices entries of width d (about 20 + 4.5 d bytes per entry); 0 for
+ * arguments outside d in 1..DQ_MAX_D, n_indices in [0, 2^31).
+ */
+size_t dq_embbag_int4_bwd_workspace_bytes(int32_t d, int64_t n_indices);
+
+/*
+ * dq_embbag_int4_bwd_sgd -- backward of dq_embbag_int4_fwd with an SGD step on
+ * binary32 master rows and re-quantization of the touched rows: the training step
+ * of "Deep Quantized Recommendation Model (DQRM)", repository page (embedding
+ * tables trained at INT4 with quantization-aware training). The pages fix no
+ * arithmetic for it; this library computes:
+ *   1. Entries: every position p of bag (t, b) with a valid id gives the entry
+ *      (key = rows of tables 0..t-1 + id, p); the entries are sorted by (key, p).
+ *   2. G (row gradient), element k: the binary64 sum of grad_out[b][t*d + k] over the
+ *      row's entries inside each window of 64 consecutive sorted entries (windows at
+ *      sorted positions 0, 64, 128, ...), summed from +0 in list order; those window
+ *      parts added from +0 in window order in binary64; rounded once to binary32.
+ *   3. master[id][k] = fma(-lr, G_k, master[id][k]) (binary32, one rounding).
+ *   4. Each touched row is quantized again from its new master values (as
+ *      dq_quantize_rows_int4 with `mode`, without row_loss/best_ij); untouched rows
+ *      keep their codes, scale/bias and master values.
+ * The result does not depend on scheduling: repeated calls give identical bits.
+ *
+ *   tables      HOST array of n_tables dq_master_table (1..DQ_MAX_TABLES)
+ *   d           1..DQ_MAX_D
+ *   indices, offsets, batch   as for dq_embbag_int4_fwd, but the offsets must be a CSR
+ *               array: offsets[0] = 0, nondecreasing, offsets[n_tables*batch] =
+ *               n_indices. Otherwise nothing is changed and DQ_FLAG_BAD_OFFSETS is
+ *               raised (checked on the device)
+ *   n_indices   number of ids, [0, 2^31); 0 is a no-op
+ *   grad_out    [batch][n_tables*d] binary32, 4-byte aligned: gradient of the lookup
+ *   lr          finite learning rate
+ *   mode        DQ_MODE_GREEDY or DQ_MODE_MINMAX for the re-quantization
+ *   workspace   device buffer, 256-byte aligned, of at least
+ *               dq_embbag_int4_bwd_workspace_bytes(d, n_indices) bytes, owned by the
+ *               caller and not in use by another call in flight; no contents kept
+ *   d_flags     device uint32 (nullable): DQ_FLAG_BAD_INDEX (invalid ids, skipped),
+ *               DQ_FLAG_BAD_OFFSETS, DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW
+ * Masters and packed tables must not overlap each other, the workspace or grad_out.
+ */
+dq_status dq_embbag_int4_bwd_sgd(const dq_master_table *tables, int32_t n_tables, int32_t d,
+                                 const int32_t *indices, const int32_t *offsets, int32_t batch,
+                                 int64_t n_indices, const float *grad_out, float lr, int32_t mode,
+                                 void *workspace, size_t workspace_bytes, uint32_t *d_flags,
+                                 void *cuda_stream);
 
 /* Static text for a status code. */
 const char *dq_status_string(dq_status s);

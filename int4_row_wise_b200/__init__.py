@@ -9,9 +9,10 @@ raises DqError (build it with `python -m int4_row_wise_b200.build`).
 
 Low-level calls with the C names:
     dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd, dq_row_l2_error,
+    dq_embbag_int4_bwd_workspace_bytes, dq_embbag_int4_bwd_sgd,
     dq_status_string, dq_last_error, dq_version
 Convenience wrappers that allocate their outputs with torch:
-    quantize_rows, dequantize_rows, embbag, row_l2_error
+    quantize_rows, dequantize_rows, embbag, row_l2_error, embbag_bwd_sgd
 """
 from __future__ import annotations
 
@@ -26,8 +27,9 @@ __all__ = [
     "DQ_FLAG_BAD_INDEX", "DQ_FLAG_BAD_OFFSETS", "DQ_FLAG_NONFINITE", "DQ_FLAG_FP16_OVERFLOW",
     "DQ_MAX_D", "DQ_MAX_TABLES", "DqError", "PackedTable", "lib_path", "load",
     "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_row_l2_error",
+    "dq_embbag_int4_bwd_workspace_bytes", "dq_embbag_int4_bwd_sgd", "MasterTable",
     "dq_status_string", "dq_last_error", "dq_version",
-    "quantize_rows", "dequantize_rows", "embbag", "row_l2_error",
+    "quantize_rows", "dequantize_rows", "embbag", "row_l2_error", "embbag_bwd_sgd",
 ]
 
 DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA = 0, 1, 2, 3
@@ -50,6 +52,11 @@ class DqError(RuntimeError):
 class _Table(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scale_bias", ctypes.c_void_p),
                 ("n_rows", ctypes.c_int64), ("codes_ld", ctypes.c_int64)]
+
+
+class _MasterTable(ctypes.Structure):
+    _fields_ = [("master", ctypes.c_void_p), ("master_ld", ctypes.c_int64), ("codes", ctypes.c_void_p),
+                ("codes_ld", ctypes.c_int64), ("scale_bias", ctypes.c_void_p), ("n_rows", ctypes.c_int64)]
 
 
 def lib_path() -> str:
@@ -75,6 +82,11 @@ def load():
             L.dq_embbag_int4_fwd.restype = ctypes.c_int
             L.dq_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp]
             L.dq_row_l2_error.restype = ctypes.c_int
+            L.dq_embbag_int4_bwd_workspace_bytes.argtypes = [i32, i64]
+            L.dq_embbag_int4_bwd_workspace_bytes.restype = ctypes.c_size_t
+            L.dq_embbag_int4_bwd_sgd.argtypes = [vp, i32, i32, vp, vp, i32, i64, vp, ctypes.c_float, i32, vp,
+                                                 ctypes.c_size_t, vp, vp]
+            L.dq_embbag_int4_bwd_sgd.restype = ctypes.c_int
             L.dq_status_string.argtypes, L.dq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
             L.dq_last_error.argtypes, L.dq_last_error.restype = [], ctypes.c_char_p
             L.dq_version.argtypes, L.dq_version.restype = [], i32
@@ -172,6 +184,40 @@ def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, o
     _check(st, "dq_embbag_int4_fwd")
 
 
+class MasterTable(NamedTuple):
+    """A trained table on the device: binary32 masters [n, master_ld] and their packed
+    form (codes uint8 [n, codes_ld], scale_bias int16 [n, 2])."""
+    master: object
+    codes: object
+    scale_bias: object
+
+
+def dq_embbag_int4_bwd_workspace_bytes(d: int, n_indices: int) -> int:
+    """C: dq_embbag_int4_bwd_workspace_bytes."""
+    return int(load().dq_embbag_int4_bwd_workspace_bytes(d, n_indices))
+
+
+def _row_stride(t) -> int:
+    return int(t.stride(0)) if t.shape[0] > 1 else int(t.shape[1])
+
+
+def dq_embbag_int4_bwd_sgd(tables: Sequence, d: int, indices, offsets, batch: int, n_indices: int, grad_out,
+                           lr: float, mode: int, workspace, workspace_bytes: int, d_flags=None,
+                           stream=None) -> None:
+    """C: dq_embbag_int4_bwd_sgd. tables: MasterTable (or (master, codes, scale_bias)) per table."""
+    arr = (_MasterTable * max(len(tables), 1))()
+    for t, tab in enumerate(tables):
+        master, codes, sb = tab[0], tab[1], tab[2]
+        if master.dim() != 2 or codes.dim() != 2:
+            raise DqError(DQ_ERR_INVALID_ARG, "master and codes must be 2-d tensors")
+        arr[t] = _MasterTable(_ptr(master), _row_stride(master), _ptr(codes), _row_stride(codes), _ptr(sb),
+                              int(master.shape[0]))
+    st = load().dq_embbag_int4_bwd_sgd(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
+                                       _ptr(offsets), batch, n_indices, _ptr(grad_out), float(lr), mode,
+                                       _ptr(workspace), workspace_bytes, _ptr(d_flags), _stream(stream))
+    _check(st, "dq_embbag_int4_bwd_sgd")
+
+
 # -------------------------------------------------------------------------
 # convenience wrappers (torch allocates the outputs on the input's device)
 # -------------------------------------------------------------------------
@@ -223,3 +269,18 @@ def row_l2_error(x, codes, scale_bias, stream=None):
     dq_row_l2_error(x, n, d, x.stride(0) if n > 1 else d, codes, codes.stride(0) if n > 1 else codes.shape[1],
                     scale_bias, err, tot, stream)
     return err, tot / max(n, 1)
+
+
+def embbag_bwd_sgd(tables: Sequence, d: int, indices, offsets, batch: int, grad_out, lr: float,
+                   mode: int = DQ_MODE_GREEDY, workspace=None, d_flags=None, stream=None):
+    """Backward of the lookup + SGD step on the masters + re-quantization of the touched
+    rows, in place. Allocates the workspace with torch unless one (uint8 CUDA tensor,
+    256-byte aligned) is given; returns it for reuse."""
+    import torch
+    n = int(indices.numel())
+    need = dq_embbag_int4_bwd_workspace_bytes(d, n)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=indices.device)
+    dq_embbag_int4_bwd_sgd(tables, d, indices, offsets, batch, n, grad_out, lr, mode, workspace,
+                           int(workspace.numel()), d_flags, stream)
+    return workspace

@@ -204,6 +204,125 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
     return launched(dq::launch_row_l2(a, sms, (cudaStream_t)cuda_stream), "row_l2_error");
 }
 
+size_t dq_embbag_int4_bwd_workspace_bytes(int32_t d, int64_t n_indices)
+{
+    if (d < 1 || d > DQ_MAX_D || n_indices < 0 || n_indices > INT32_MAX)
+        return 0;
+    return dq::bwd_layout(n_indices, d).total;
+}
+
+dq_status dq_embbag_int4_bwd_sgd(const dq_master_table *tables, int32_t n_tables, int32_t d,
+                                 const int32_t *indices, const int32_t *offsets, int32_t batch, int64_t n_indices,
+                                 const float *grad_out, float lr, int32_t mode, void *workspace,
+                                 size_t workspace_bytes, uint32_t *d_flags, void *cuda_stream)
+{
+    if (n_tables < 1 || n_tables > DQ_MAX_TABLES)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables = %d outside [1, %d]", n_tables, DQ_MAX_TABLES);
+    if (!tables)
+        return fail(DQ_ERR_INVALID_ARG, "tables must be non-NULL");
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (batch < 0)
+        return fail(DQ_ERR_INVALID_ARG, "batch = %d < 0", batch);
+    if ((int64_t)n_tables * batch + 1 > INT32_MAX)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables * batch + 1 offsets exceed int32 indexing");
+    if (n_indices < 0 || n_indices > INT32_MAX)
+        return fail(DQ_ERR_INVALID_ARG, "n_indices = %lld outside [0, 2^31)", (long long)n_indices);
+    if (batch == 0 && n_indices != 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_indices = %lld with batch = 0", (long long)n_indices);
+    if (mode != DQ_MODE_GREEDY && mode != DQ_MODE_MINMAX)
+        return fail(DQ_ERR_INVALID_ARG, "mode = %d is neither DQ_MODE_GREEDY nor DQ_MODE_MINMAX", mode);
+    if (!(lr - lr == 0.0f))
+        return fail(DQ_ERR_INVALID_ARG, "lr is not finite");
+    dq::RequantArgs r;
+    memset(&r, 0, sizeof r);
+    int64_t total = 0;
+    for (int t = 0; t < n_tables; ++t) {
+        const dq_master_table &tb = tables[t];
+        if (tb.n_rows < 0)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].n_rows = %lld < 0", t, (long long)tb.n_rows);
+        if (tb.master_ld < d)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].master_ld = %lld < d = %d", t, (long long)tb.master_ld, d);
+        if (tb.codes_ld < (d + 1) / 2)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].codes_ld = %lld < (d+1)/2 = %d", t,
+                        (long long)tb.codes_ld, (d + 1) / 2);
+        if (tb.n_rows > 0 && (!tb.master || !tb.codes || !tb.scale_bias))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: master, codes and scale_bias must be non-NULL", t);
+        if ((reinterpret_cast<uintptr_t>(tb.master) & 3) || (reinterpret_cast<uintptr_t>(tb.scale_bias) & 1))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: master must be 4-byte and scale_bias 2-byte aligned", t);
+        r.tabs.master[t] = tb.master;
+        r.tabs.master_ld[t] = tb.master_ld;
+        r.tabs.codes[t] = tb.codes;
+        r.tabs.codes_ld[t] = tb.codes_ld;
+        r.tabs.scale_bias[t] = tb.scale_bias;
+        r.tabs.key_base[t] = (uint32_t)total;
+        total += tb.n_rows;
+        if (total > (int64_t)UINT32_MAX - 1)
+            return fail(DQ_ERR_INVALID_ARG, "the tables hold more than 2^32 - 2 rows in all");
+    }
+    r.tabs.key_base[n_tables] = (uint32_t)total;
+    if (n_indices == 0)
+        return ok();
+    if (!indices || !offsets || !grad_out)
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and grad_out must be non-NULL when n_indices > 0");
+    if (reinterpret_cast<uintptr_t>(grad_out) & 3)
+        return fail(DQ_ERR_INVALID_ARG, "grad_out must be 4-byte aligned");
+    const dq::BwdLayout L = dq::bwd_layout(n_indices, d);
+    if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return fail(DQ_ERR_INVALID_ARG, "workspace must be a non-NULL, 256-byte aligned device buffer");
+    if (workspace_bytes < L.total)
+        return fail(DQ_ERR_INVALID_ARG, "workspace_bytes = %zu < %zu needed (dq_embbag_int4_bwd_workspace_bytes)",
+                    workspace_bytes, L.total);
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    char *ws = static_cast<char *>(workspace);
+    dq::BwdArgs a;
+    memset(&a, 0, sizeof a);
+    a.T = n_tables;
+    a.d = d;
+    a.batch = batch;
+    a.n = n_indices;
+    a.indices = indices;
+    a.offsets = offsets;
+    a.grad = grad_out;
+    memcpy(a.key_base, r.tabs.key_base, sizeof a.key_base);
+    a.div = dq::make_batch_div((uint32_t)batch);
+    a.hdr = reinterpret_cast<uint32_t *>(ws + L.hdr);
+    a.keys[0] = reinterpret_cast<uint32_t *>(ws + L.keys0);
+    a.keys[1] = reinterpret_cast<uint32_t *>(ws + L.keys1);
+    a.bags[0] = reinterpret_cast<int32_t *>(ws + L.bags0);
+    a.bags[1] = reinterpret_cast<int32_t *>(ws + L.bags1);
+    a.hist = reinterpret_cast<uint32_t *>(ws + L.hist);
+    a.totals = reinterpret_cast<uint32_t *>(ws + L.totals);
+    a.partials = reinterpret_cast<double *>(ws + L.partials);
+    a.list = reinterpret_cast<uint32_t *>(ws + L.list);
+    a.grad_rows = reinterpret_cast<float *>(ws + L.grad_rows);
+    a.grad_ld = L.grad_ld;
+    a.flags = d_flags;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    cudaError_t e = cudaMemsetAsync(a.hdr, 0, 256, stream);
+    if (e != cudaSuccess)
+        return fail(DQ_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    e = dq::launch_bwd_sort_reduce(a, sms, stream);
+    if (e != cudaSuccess)
+        return launched(e, "embbag backward");
+    r.n_tables = n_tables;
+    r.d = d;
+    r.list = a.list;
+    r.count = a.hdr + 1;
+    r.bad = a.hdr;
+    r.grad_rows = a.grad_rows;
+    r.grad_ld = a.grad_ld;
+    r.lr = lr;
+    r.flags = d_flags;
+    const int64_t max_rows = n_indices < total ? n_indices : total;
+    return launched(dq::launch_requant(r, max_rows, mode, sms, stream), "embbag backward re-quantization");
+}
+
 const char *dq_status_string(dq_status s)
 {
     switch (s) {

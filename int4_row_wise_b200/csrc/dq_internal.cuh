@@ -68,6 +68,60 @@ struct BagArgs {
     BatchDiv div;
 };
 
+// Master and packed tables of the bag backward, passed by value (about 2.8 KB of
+// parameter space). Row id of table t has the global key key_base[t] + id;
+// key_base[n_tables] is the total row count and marks invalid entries.
+struct RequantTables {
+    float *master[DQ_MAX_TABLES];
+    int64_t master_ld[DQ_MAX_TABLES];
+    uint8_t *codes[DQ_MAX_TABLES];
+    int64_t codes_ld[DQ_MAX_TABLES];
+    uint16_t *scale_bias[DQ_MAX_TABLES];
+    uint32_t key_base[DQ_MAX_TABLES + 1];
+};
+
+// Re-quantization of the rows listed by the bag backward, with the SGD step.
+struct RequantArgs {
+    RequantTables tabs;
+    int n_tables, d;
+    const uint32_t *list;      // global keys of the listed rows
+    const uint32_t *count;     // number of listed rows (device)
+    const uint32_t *bad;       // nonzero: the offsets were rejected, nothing to do
+    const float *grad_rows;    // G of listed row i at grad_rows + i * grad_ld
+    int64_t grad_ld;
+    float lr;
+    uint32_t *flags;
+};
+
+// The bag backward's sort and reduction. The workspace pointers are carved from
+// the caller's buffer (bwd_layout).
+struct BwdArgs {
+    int T, d, batch;
+    int64_t n;                 // number of indices = entries
+    const int32_t *indices;
+    const int32_t *offsets;
+    const float *grad;         // [batch][T * d]
+    uint32_t key_base[DQ_MAX_TABLES + 1];
+    BatchDiv div;
+    uint32_t *hdr;             // [0] offsets rejected, [1] rows listed
+    uint32_t *keys[2];
+    int32_t *bags[2];
+    uint32_t *hist;            // [256][tiles]
+    uint32_t *totals;          // [256]
+    double *partials;          // [windows][2][d]
+    uint32_t *list;            // [entries]
+    float *grad_rows;          // [entries][grad_ld]
+    int64_t grad_ld;
+    uint32_t *flags;
+};
+
+// Byte offsets of the pieces of the backward's workspace (each 256-byte aligned).
+struct BwdLayout {
+    size_t hdr, keys0, keys1, bags0, bags1, hist, totals, partials, list, grad_rows, total;
+    int64_t tiles, windows, grad_ld;
+};
+BwdLayout bwd_layout(int64_t n, int d);
+
 inline BatchDiv make_batch_div(uint32_t dvs)
 {
     uint32_t l = 0;
@@ -90,6 +144,8 @@ cudaError_t launch_quantize(const QuantArgs &a, int mode, int num_sms, cudaStrea
 cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_requant(const RequantArgs &a, int64_t max_rows, int mode, int num_sms, cudaStream_t stream);
 
 __device__ __forceinline__ void raise_flag(uint32_t *flags, uint32_t bit)
 {

@@ -281,21 +281,46 @@ __device__ __forceinline__ void greedy_walk(const float2 (&xp)[H], int kbase, in
     }
 }
 
+// Where a row of the plain kernel lives: row r of the caller's arrays. The pointers
+// are formed where they are used, so nothing but r stays live across the search.
+struct PlainRow {
+    const QuantArgs &a;
+    int64_t r;
+    __device__ __forceinline__ const float *x() const { return a.x + r * a.ld; }
+    __device__ __forceinline__ uint8_t *codes() const { return a.codes + r * a.codes_ld; }
+    __device__ __forceinline__ uint16_t *scale_bias() const { return a.scale_bias + 2 * r; }
+    __device__ __forceinline__ float *loss() const { return a.row_loss ? a.row_loss + r : nullptr; }
+    __device__ __forceinline__ uint8_t *best_ij() const { return a.best_ij ? a.best_ij + 2 * r : nullptr; }
+};
+
+// A row listed by the bag backward: entry i names master row id of table t and its
+// gradient row G_i; the master row is first moved to fma(-lr, G, w) (and written back).
+struct ListedRow {
+    const RequantArgs &a;
+    int64_t i;
+    int t;
+    int64_t id;
+    __device__ __forceinline__ const float *x() const { return a.tabs.master[t] + id * a.tabs.master_ld[t]; }
+    __device__ __forceinline__ float *x_out() const { return a.tabs.master[t] + id * a.tabs.master_ld[t]; }
+    __device__ __forceinline__ const float *grad() const { return a.grad_rows + i * a.grad_ld; }
+    __device__ __forceinline__ uint8_t *codes() const { return a.tabs.codes[t] + id * a.tabs.codes_ld[t]; }
+    __device__ __forceinline__ uint16_t *scale_bias() const { return a.tabs.scale_bias[t] + 2 * id; }
+    __device__ __forceinline__ float *loss() const { return nullptr; }
+    __device__ __forceinline__ uint8_t *best_ij() const { return nullptr; }
+};
+
 // One row per W lanes; M elements per lane; FULL: d == M * W (no padding);
-// VEC: 16-byte loads of x and vector stores of the codes are aligned.
-template <int M, int W, bool FULL, bool VEC>
-__global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, const int greedy)
+// VEC: 16-byte loads of x and vector stores of the codes are aligned. SGD: the row is
+// x + (-lr) * grad, rounded once per element, and is stored back before the search.
+template <int M, int W, bool FULL, bool VEC, bool SGD, class Row>
+__device__ __forceinline__ void quantize_one(const Row &src, const int d, const bool active, const int greedy,
+                                             const float lr, uint32_t *flags)
 {
     constexpr bool HAS_Y = M > 1;
     constexpr int H = HAS_Y ? M / 2 : 1;
     const int sub = threadIdx.x & (W - 1);
-    int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
-    const bool active = row < a.n;
-    if (!active)
-        row = a.n - 1;  // idle lanes shadow the last row so the warp stays converged
-    const int d = a.d;
     const int kbase = sub * M;
-    const float *xr = a.x + row * a.ld + kbase;
+    const float *xr = src.x() + kbase;
 
     // the lane's M elements: element k in xp[k].x (k < H) or xp[k - H].y
     float2 xp[H];
@@ -303,7 +328,17 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
         float v[M];
 #pragma unroll
         for (int m = 0; m < M; m += 4) {
-            const float4 q4 = __ldg(reinterpret_cast<const float4 *>(xr + m));
+            float4 q4 = SGD ? *reinterpret_cast<const float4 *>(xr + m)
+                            : __ldg(reinterpret_cast<const float4 *>(xr + m));
+            if constexpr (SGD) {
+                const float4 g4 = __ldg(reinterpret_cast<const float4 *>(src.grad() + kbase + m));
+                q4.x = __fmaf_rn(-lr, g4.x, q4.x);
+                q4.y = __fmaf_rn(-lr, g4.y, q4.y);
+                q4.z = __fmaf_rn(-lr, g4.z, q4.z);
+                q4.w = __fmaf_rn(-lr, g4.w, q4.w);
+                if (active)
+                    *reinterpret_cast<float4 *>(src.x_out() + kbase + m) = q4;
+            }
             v[m] = q4.x;
             v[m + 1] = q4.y;
             v[m + 2] = q4.z;
@@ -315,8 +350,23 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
     } else {
 #pragma unroll
         for (int h = 0; h < H; ++h) {
-            xp[h].x = valid_x<H, HAS_Y, FULL>(kbase, h, d) ? __ldg(xr + h) : 0.0f;
-            xp[h].y = valid_y<H, HAS_Y, FULL>(kbase, h, d) ? __ldg(xr + h + H) : 0.0f;
+            const bool vx = valid_x<H, HAS_Y, FULL>(kbase, h, d), vy = valid_y<H, HAS_Y, FULL>(kbase, h, d);
+            xp[h].x = vx ? (SGD ? xr[h] : __ldg(xr + h)) : 0.0f;
+            xp[h].y = vy ? (SGD ? xr[h + H] : __ldg(xr + h + H)) : 0.0f;
+            if constexpr (SGD) {
+                const float *gr = src.grad() + kbase;
+                float *xo = src.x_out() + kbase;
+                if (vx) {
+                    xp[h].x = __fmaf_rn(-lr, __ldg(gr + h), xp[h].x);
+                    if (active)
+                        xo[h] = xp[h].x;
+                }
+                if (vy) {
+                    xp[h].y = __fmaf_rn(-lr, __ldg(gr + h + H), xp[h].y);
+                    if (active)
+                        xo[h + H] = xp[h].y;
+                }
+            }
         }
     }
 
@@ -385,7 +435,7 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
     if (!active)
         return;
 
-    uint8_t *cr = a.codes + row * a.codes_ld + kbase / 2;
+    uint8_t *cr = src.codes() + kbase / 2;
     if constexpr (VEC && M >= 2) {
         if constexpr (M == 32) {
             uint4 w;
@@ -413,20 +463,70 @@ __global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, c
                 cr[m] = packed[m];
     }
     if (sub == 0) {
-        a.scale_bias[2 * row] = __half_as_ushort(s16);
-        a.scale_bias[2 * row + 1] = __half_as_ushort(b16);
-        if (a.row_loss)
-            a.row_loss[row] = lbest;
-        if (a.best_ij) {
-            a.best_ij[2 * row] = (uint8_t)bi;
-            a.best_ij[2 * row + 1] = (uint8_t)bj;
+        uint16_t *sb = src.scale_bias();
+        sb[0] = __half_as_ushort(s16);
+        sb[1] = __half_as_ushort(b16);
+        if (float *lp = src.loss())
+            *lp = lbest;
+        if (uint8_t *ij = src.best_ij()) {
+            ij[0] = (uint8_t)bi;
+            ij[1] = (uint8_t)bj;
         }
         if (isinf(S) || isinf(B))
-            raise_flag(a.flags, DQ_FLAG_FP16_OVERFLOW);
+            raise_flag(flags, DQ_FLAG_FP16_OVERFLOW);
     }
     if (nonfinite)
-        raise_flag(a.flags, DQ_FLAG_NONFINITE);
+        raise_flag(flags, DQ_FLAG_NONFINITE);
 }
+
+template <int M, int W, bool FULL, bool VEC>
+__global__ void __launch_bounds__(128) quantize_rows_kernel(const QuantArgs a, const int greedy)
+{
+    int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
+    const bool active = row < a.n;
+    if (!active)
+        row = a.n - 1;  // idle lanes shadow the last row so the warp stays converged
+    quantize_one<M, W, FULL, VEC, false>(PlainRow{a, row}, a.d, active, greedy, 0.0f, a.flags);
+}
+
+// Table of a global row key: the last table whose first key is <= key.
+__device__ __forceinline__ int table_of_key(const RequantTables &tabs, int n_tables, uint32_t key)
+{
+    int lo = 0, hi = n_tables;  // tabs.key_base[lo] <= key < tabs.key_base[hi] (key_base[n_tables] = total)
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tabs.key_base[mid] <= key)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Re-quantization of the rows the bag backward listed, with their SGD step fused in.
+// Grid-stride over the list (its length is known on the device only); the loop
+// bound is warp-uniform, so the row's lanes stay converged for the shuffles.
+template <int M, int W, bool FULL, bool VEC>
+__global__ void __launch_bounds__(128) requant_rows_kernel(const RequantArgs a, const int greedy)
+{
+    if (*a.bad)
+        return;
+    const int64_t count = *a.count;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t first = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); first < count * W;
+         first += stride) {
+        int64_t i = (first + (threadIdx.x & 31)) / W;
+        const bool active = i < count;
+        if (!active)
+            i = count - 1;
+        const uint32_t key = a.list[i];
+        const int t = table_of_key(a.tabs, a.n_tables, key);
+        quantize_one<M, W, FULL, VEC, true>(ListedRow{a, i, t, (int64_t)(key - a.tabs.key_base[t])}, a.d, active,
+                                            greedy, a.lr, a.flags);
+    }
+}
+
+
 
 template <int M, int W>
 cudaError_t launch_mw(const QuantArgs &a, int greedy, cudaStream_t stream)
@@ -450,7 +550,58 @@ cudaError_t launch_mw(const QuantArgs &a, int greedy, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+template <int M, int W>
+cudaError_t launch_requant_mw(const RequantArgs &a, int64_t max_rows, int greedy, int num_sms,
+                              cudaStream_t stream)
+{
+    constexpr int kBlock = 128;
+    // grid-stride over at most max_rows rows: enough blocks to fill every SM a few times
+    const int64_t need = (max_rows * W + kBlock - 1) / kBlock;
+    const int64_t cap = (int64_t)num_sms * 16;
+    const unsigned grid = (unsigned)(need < cap ? need : cap);
+    const bool full = a.d == M * W;
+    bool vec = full && (M % 4 == 0) && (a.grad_ld % 4 == 0) &&
+               (reinterpret_cast<uintptr_t>(a.grad_rows) & 15) == 0;
+    for (int t = 0; t < a.n_tables && vec; ++t)
+        vec = a.tabs.master_ld[t] % 4 == 0 && (reinterpret_cast<uintptr_t>(a.tabs.master[t]) & 15) == 0 &&
+              a.tabs.codes_ld[t] % ((M + 1) / 2) == 0 &&
+              reinterpret_cast<uintptr_t>(a.tabs.codes[t]) % ((M + 1) / 2) == 0;
+    if (vec) {
+        if constexpr (M % 4 == 0)
+            requant_rows_kernel<M, W, true, true><<<grid, kBlock, 0, stream>>>(a, greedy);
+    } else if (full) {
+        requant_rows_kernel<M, W, true, false><<<grid, kBlock, 0, stream>>>(a, greedy);
+    } else {
+        requant_rows_kernel<M, W, false, false><<<grid, kBlock, 0, stream>>>(a, greedy);
+    }
+    return cudaGetLastError();
+}
+
 } // namespace
+
+cudaError_t launch_requant(const RequantArgs &a, int64_t max_rows, int mode, int num_sms, cudaStream_t stream)
+{
+    if (max_rows <= 0)
+        return cudaSuccess;
+    int p = 1;
+    while (p < a.d)
+        p <<= 1;
+    const int greedy = mode == DQ_MODE_GREEDY;
+    switch (p) {
+    case 1: return launch_requant_mw<1, 1>(a, max_rows, greedy, num_sms, stream);
+    case 2: return launch_requant_mw<2, 1>(a, max_rows, greedy, num_sms, stream);
+    case 4: return launch_requant_mw<4, 1>(a, max_rows, greedy, num_sms, stream);
+    case 8: return launch_requant_mw<8, 1>(a, max_rows, greedy, num_sms, stream);
+    case 16: return launch_requant_mw<16, 1>(a, max_rows, greedy, num_sms, stream);
+    case 32: return launch_requant_mw<16, 2>(a, max_rows, greedy, num_sms, stream);
+    case 64: return launch_requant_mw<16, 4>(a, max_rows, greedy, num_sms, stream);
+    case 128: return launch_requant_mw<16, 8>(a, max_rows, greedy, num_sms, stream);
+    case 256: return launch_requant_mw<16, 16>(a, max_rows, greedy, num_sms, stream);
+    case 512: return launch_requant_mw<16, 32>(a, max_rows, greedy, num_sms, stream);
+    case 1024: return launch_requant_mw<32, 32>(a, max_rows, greedy, num_sms, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_quantize(const QuantArgs &a, int mode, int /*num_sms*/, cudaStream_t stream)
 {

@@ -113,3 +113,48 @@ def test_library_sources_allocate_nothing():
         src = open(path).read()
         for call in ("cudaMalloc", "cudaFree", "cudaHostAlloc", "cudaMallocHost", "malloc(", "new "):
             assert call not in src, (path, call)
+
+
+def _masters(*specs):
+    arr = (dq._MasterTable * max(len(specs), 1))(*[dq._MasterTable(*s) for s in specs])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+_M, _C, _S = 1 << 20, 1 << 22, 1 << 24  # placeholder device addresses (never dereferenced)
+
+
+@pytest.mark.parametrize("tabspec,T,d,batch,n,lr,mode,ws,wsb,msg", [
+    ([(_M, 16, _C, 8, _S, 10)], 0, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "n_tables = 0"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 0, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "d = 0"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, -1, 8, 0.1, 0, 1 << 26, 1 << 30, "batch"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 4, -1, 0.1, 0, 1 << 26, 1 << 30, "n_indices"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 0, 3, 0.1, 0, 1 << 26, 1 << 30, "batch = 0"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 5, 1 << 26, 1 << 30, "mode"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 4, 8, float("inf"), 0, 1 << 26, 1 << 30, "lr"),
+    ([(_M, 15, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "master_ld"),
+    ([(_M, 16, _C, 7, _S, 10)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "codes_ld"),
+    ([(_M, 16, _C, 8, _S, -2)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "n_rows"),
+    ([(None, 16, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "non-NULL"),
+    ([(_M + 2, 16, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30, "aligned"),
+    ([(_M, 16, _C, 8, _S, 1 << 31), (_M, 16, _C, 8, _S, 1 << 31)], 2, 16, 4, 8, 0.1, 0, 1 << 26, 1 << 30,
+     "2^32 - 2"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 0, (1 << 26) + 16, 1 << 30, "256-byte"),
+    ([(_M, 16, _C, 8, _S, 10)], 1, 16, 4, 8, 0.1, 0, 1 << 26, 100, "workspace_bytes"),
+])
+def test_embbag_bwd_rejects(L, tabspec, T, d, batch, n, lr, mode, ws, wsb, msg):
+    p, keep = _masters(*tabspec)
+    idx, off, g = 1 << 27, 1 << 28, 1 << 29
+    st = L.dq_embbag_int4_bwd_sgd(p, T, d, idx, off, batch, n, g, lr, mode, ws, wsb, None, None)
+    assert st == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
+def test_embbag_bwd_no_entries_is_a_noop_and_workspace_size(L):
+    p, keep = _masters((_M, 16, _C, 8, _S, 10))
+    assert L.dq_embbag_int4_bwd_sgd(p, 1, 16, None, None, 4, 0, None, 0.1, 0, None, 0, None, None) == dq.DQ_OK
+    assert dq.dq_embbag_int4_bwd_workspace_bytes(16, -1) == 0
+    assert dq.dq_embbag_int4_bwd_workspace_bytes(0, 10) == 0
+    small, big = dq.dq_embbag_int4_bwd_workspace_bytes(64, 1000), dq.dq_embbag_int4_bwd_workspace_bytes(64, 10 ** 6)
+    assert small % 256 == 0 and big % 256 == 0
+    # keys, bags (twice each), list: 20 B; G rows: 4 d B; window parts: d / 4 B per entry
+    assert 10 ** 6 * (20 + 4 * 64 + 64 // 4) <= big <= 10 ** 6 * (20 + 4 * 64 + 64 // 4) + 10 ** 6
