@@ -225,6 +225,29 @@ dq_status dq_embbag_int4_bwd_sgd(const dq_master_table *tables, int32_t n_tables
                                  void *workspace, size_t workspace_bytes, uint32_t *d_flags,
                                  void *cuda_stream);
 
+/*
+ * dq_embbag_int4_bwd_sgd_noalloc -- dq_embbag_int4_bwd_sgd without a caller
+ * workspace, for callers that cannot allocate device memory (a plugin inside a host
+ * program that owns the allocator, a process under a fixed memory budget, a server
+ * that must not grow its device footprint). The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Its scratch is one static device array of DQ_BWD_STATIC_SCRATCH_BYTES (32 MiB),
+ * held by every GPU that loads the library until the process exits. The call
+ * allocates nothing. Arguments and results are those of dq_embbag_int4_bwd_sgd; a
+ * call whose dq_embbag_int4_bwd_workspace_bytes(d, n_indices) exceeds the array is
+ * rejected with DQ_ERR_INVALID_ARG (about 110,000 entries at d = 64).
+ * The first call on a device looks up the array's device address there (once per
+ * device), so make it before any stream capture. All calls share the array: calls
+ * whose work overlaps on the GPU (several streams or host threads) race and must be
+ * serialized by the caller. Each call clears what must start at zero itself.
+ */
+#define DQ_BWD_STATIC_SCRATCH_BYTES (32u << 20)
+dq_status dq_embbag_int4_bwd_sgd_noalloc(const dq_master_table *tables, int32_t n_tables, int32_t d,
+                                         const int32_t *indices, const int32_t *offsets, int32_t batch,
+                                         int64_t n_indices, const float *grad_out, float lr, int32_t mode,
+                                         uint32_t *d_flags, void *cuda_stream);
+
 /* Static text for a status code. */
 const char *dq_status_string(dq_status s);
 

@@ -9,7 +9,7 @@ raises DqError (build it with `python -m int4_row_wise_b200.build`).
 
 Low-level calls with the C names:
     dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd, dq_row_l2_error,
-    dq_embbag_int4_bwd_workspace_bytes, dq_embbag_int4_bwd_sgd,
+    dq_embbag_int4_bwd_workspace_bytes, dq_embbag_int4_bwd_sgd, dq_embbag_int4_bwd_sgd_noalloc,
     dq_status_string, dq_last_error, dq_version
 Convenience wrappers that allocate their outputs with torch:
     quantize_rows, dequantize_rows, embbag, row_l2_error, embbag_bwd_sgd
@@ -28,6 +28,7 @@ __all__ = [
     "DQ_MAX_D", "DQ_MAX_TABLES", "DqError", "PackedTable", "lib_path", "load",
     "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_row_l2_error",
     "dq_embbag_int4_bwd_workspace_bytes", "dq_embbag_int4_bwd_sgd", "MasterTable",
+    "dq_embbag_int4_bwd_sgd_noalloc", "DQ_BWD_STATIC_SCRATCH_BYTES",
     "dq_status_string", "dq_last_error", "dq_version",
     "quantize_rows", "dequantize_rows", "embbag", "row_l2_error", "embbag_bwd_sgd",
 ]
@@ -36,6 +37,7 @@ DQ_OK, DQ_ERR_INVALID_ARG, DQ_ERR_UNSUPPORTED, DQ_ERR_CUDA = 0, 1, 2, 3
 DQ_MODE_GREEDY, DQ_MODE_MINMAX = 0, 1
 DQ_FLAG_BAD_INDEX, DQ_FLAG_BAD_OFFSETS, DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW = 1, 2, 4, 8
 DQ_MAX_D, DQ_MAX_TABLES = 1024, 64
+DQ_BWD_STATIC_SCRATCH_BYTES = 32 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdq.so")
@@ -87,6 +89,9 @@ def load():
             L.dq_embbag_int4_bwd_sgd.argtypes = [vp, i32, i32, vp, vp, i32, i64, vp, ctypes.c_float, i32, vp,
                                                  ctypes.c_size_t, vp, vp]
             L.dq_embbag_int4_bwd_sgd.restype = ctypes.c_int
+            L.dq_embbag_int4_bwd_sgd_noalloc.argtypes = [vp, i32, i32, vp, vp, i32, i64, vp, ctypes.c_float, i32,
+                                                         vp, vp]
+            L.dq_embbag_int4_bwd_sgd_noalloc.restype = ctypes.c_int
             L.dq_status_string.argtypes, L.dq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
             L.dq_last_error.argtypes, L.dq_last_error.restype = [], ctypes.c_char_p
             L.dq_version.argtypes, L.dq_version.restype = [], i32
@@ -216,6 +221,29 @@ def dq_embbag_int4_bwd_sgd(tables: Sequence, d: int, indices, offsets, batch: in
                                        _ptr(offsets), batch, n_indices, _ptr(grad_out), float(lr), mode,
                                        _ptr(workspace), workspace_bytes, _ptr(d_flags), _stream(stream))
     _check(st, "dq_embbag_int4_bwd_sgd")
+
+
+def _master_array(tables):
+    arr = (_MasterTable * max(len(tables), 1))()
+    for t, tab in enumerate(tables):
+        master, codes, sb = tab[0], tab[1], tab[2]
+        if master.dim() != 2 or codes.dim() != 2:
+            raise DqError(DQ_ERR_INVALID_ARG, "master and codes must be 2-d tensors")
+        arr[t] = _MasterTable(_ptr(master), _row_stride(master), _ptr(codes), _row_stride(codes), _ptr(sb),
+                              int(master.shape[0]))
+    return arr
+
+
+def dq_embbag_int4_bwd_sgd_noalloc(tables: Sequence, d: int, indices, offsets, batch: int, n_indices: int,
+                                   grad_out, lr: float, mode: int, d_flags=None, stream=None) -> None:
+    """C: dq_embbag_int4_bwd_sgd_noalloc -- the backward on the library's static device
+    scratch (DQ_BWD_STATIC_SCRATCH_BYTES), for callers that cannot allocate device
+    memory. Calls that overlap on the GPU race on that scratch."""
+    arr = _master_array(tables)
+    st = load().dq_embbag_int4_bwd_sgd_noalloc(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
+                                               _ptr(offsets), batch, n_indices, _ptr(grad_out), float(lr), mode,
+                                               _ptr(d_flags), _stream(stream))
+    _check(st, "dq_embbag_int4_bwd_sgd_noalloc")
 
 
 # -------------------------------------------------------------------------

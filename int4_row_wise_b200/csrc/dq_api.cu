@@ -75,6 +75,13 @@ dq_status launched(cudaError_t e, const char *what)
 
 } // namespace
 
+namespace dq {
+void set_last_error(const char *msg)
+{
+    g_last_error = msg;
+}
+} // namespace dq
+
 extern "C" {
 
 dq_status dq_quantize_rows_int4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, uint8_t *codes,

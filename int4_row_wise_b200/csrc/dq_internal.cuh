@@ -147,6 +147,9 @@ cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_requant(const RequantArgs &a, int64_t max_rows, int mode, int num_sms, cudaStream_t stream);
 
+// Sets the calling thread's dq_last_error() text (for entry points outside dq_api.cu).
+void set_last_error(const char *msg);
+
 __device__ __forceinline__ void raise_flag(uint32_t *flags, uint32_t bit)
 {
     if (flags)
