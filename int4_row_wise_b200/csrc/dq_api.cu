@@ -306,6 +306,7 @@ dq_status dq_embbag_int4_bwd_sgd(const dq_master_table *tables, int32_t n_tables
     a.hist = reinterpret_cast<uint32_t *>(ws + L.hist);
     a.totals = reinterpret_cast<uint32_t *>(ws + L.totals);
     a.partials = reinterpret_cast<double *>(ws + L.partials);
+    a.span_slot = reinterpret_cast<uint32_t *>(ws + L.span_slot);
     a.list = reinterpret_cast<uint32_t *>(ws + L.list);
     a.grad_rows = reinterpret_cast<float *>(ws + L.grad_rows);
     a.grad_ld = L.grad_ld;

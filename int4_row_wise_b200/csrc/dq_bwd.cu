@@ -16,17 +16,19 @@
 // scheduling, so the updated masters and their codes are reproducible.
 //
 // Kernels, in stream order:
-//   bwd_keys_kernel      one lane per bag: writes (key, bag) of each of its entries;
+//   bwd_keys_kernel      one lane (or warp) per bag: writes (key, bag) of its entries;
 //                        checks that offsets are a CSR array (else nothing changes)
 //   radix_hist_kernel    LSD radix sort, 8-bit digits, ceil(bits(total rows) / 8)
 //   radix_scan_kernel    passes of three kernels each: per-tile digit counts,
 //   radix_scatter_kernel their digit-major exclusive scan, and a stable scatter
 //                        (warp-striped tiles ranked with ballots, no atomics)
-//   bwd_window_kernel    one warp per window: sums each row's part in binary64;
-//                        a row wholly inside the window gets its G and a list slot,
-//                        a row crossing a window edge leaves a binary64 part
-//   bwd_span_kernel      one warp per row that spans windows: adds its parts in
-//                        window order and lists it
+//   bwd_window_kernel    one warp per window: stages the entries' gradient rows in
+//                        shared memory (cp.async, all in flight), sums each row's
+//                        part in binary64; lists every row that ends in the window
+//                        (with its G when the row lies wholly inside it); a row
+//                        crossing a window edge leaves a binary64 part
+//   bwd_span_kernel      one warp per (spanning row, 32 elements): adds its parts in
+//                        window order
 // Every loop is bounded by sizes known at launch; no kernel waits on another.
 #include "dq_internal.cuh"
 
@@ -38,7 +40,6 @@ constexpr int kSortThreads = 256;
 constexpr int kSortItems = 8;
 constexpr int kTile = kSortThreads * kSortItems;  // entries per sort tile
 constexpr int kDigits = 256;
-constexpr int kRedThreads = 256;                  // 8 warps per block in the reductions
 
 // Lanes of the warp whose 8-bit digit equals this lane's (only lanes with ok set).
 __device__ __forceinline__ unsigned digit_peers(uint32_t dg, bool ok)
@@ -87,20 +88,26 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t *w
 // entries
 // ---------------------------------------------------------------------------
 
+// One lane per bag (short bags) or one warp per bag (WARP: bags of 8 or more ids on
+// average, so the reads of indices and the writes of the entries are coalesced).
+template <bool WARP>
 __global__ void __launch_bounds__(256) bwd_keys_kernel(const BwdArgs a)
 {
     const int64_t G = (int64_t)a.T * a.batch;
     const uint32_t sentinel = a.key_base[a.T];
     bool bad = false, bad_id = false;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < G; g += stride) {
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t per = WARP ? 32 : 1;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x / per;
+    const int lane = WARP ? (int)(threadIdx.x & 31) : 0;
+    for (int64_t g = tid / per; g < G; g += stride) {
         int64_t p0 = a.offsets[g], p1 = a.offsets[g + 1];
         bad |= p1 < p0;
         p0 = p0 < 0 ? 0 : (p0 > a.n ? a.n : p0);  // keep every write inside the entry arrays
         p1 = p1 < p0 ? p0 : (p1 > a.n ? a.n : p1);
         const int t = (int)div_batch((uint32_t)g, a.div);
         const uint32_t base = a.key_base[t], rows = a.key_base[t + 1] - base;
-        for (int64_t p = p0; p < p1; ++p) {
+        for (int64_t p = p0 + lane; p < p1; p += per) {
             const int32_t id = __ldg(a.indices + p);
             const bool ok = id >= 0 && (uint32_t)id < rows;
             bad_id |= !ok;
@@ -108,7 +115,7 @@ __global__ void __launch_bounds__(256) bwd_keys_kernel(const BwdArgs a)
             a.bags[0][p] = (int32_t)g;
         }
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0)
+    if (tid == 0)
         bad |= a.offsets[0] != 0 || (int64_t)a.offsets[G] != a.n;
     if (bad) {
         atomicOr(a.hdr, 1u);
@@ -238,240 +245,391 @@ __global__ void __launch_bounds__(kSortThreads) radix_scatter_kernel(const uint3
 // reductions
 // ---------------------------------------------------------------------------
 
-// The lane's EPL elements [lane * EPL, lane * EPL + EPL) of a binary32 row (0 past d).
-template <int EPL, bool VEC>
-__device__ __forceinline__ void load_elems(const float *row, int lane, int d, float (&v)[EPL])
+constexpr uint32_t kNoSpan = 0xffffffffu;
+
+constexpr int kWinWarps = 4;      // warps per block in bwd_window_kernel
+constexpr int kChunk = 8;         // at most this many windows per block iteration
+constexpr int kStageFloats = 1024; // 4 KB per stage: 32 / EPL rows (at least 1) of 32 * EPL floats
+
+// L2 policy for the gradient rows: keep them (every bag's row is read once per id of
+// the bag), while the G rows and parts written alongside stream past (st.global.cs).
+__device__ __forceinline__ uint64_t evict_last_policy()
 {
-    const int k0 = lane * EPL;
-    if constexpr (VEC) {
-#pragma unroll
-        for (int e = 0; e < EPL; e += 4) {
-            const float4 q = k0 + e < d ? __ldg(reinterpret_cast<const float4 *>(row + k0 + e))
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-            v[e] = q.x;
-            v[e + 1] = q.y;
-            v[e + 2] = q.z;
-            v[e + 3] = q.w;
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, uint64_t policy)
+{
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;\n" ::"r"(d), "l"(src), "l"(policy));
+}
+
+__device__ __forceinline__ void cp_async4(void *dst, const void *src, uint64_t policy)
+{
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global.L2::cache_hint [%0], [%1], 4, %2;\n" ::"r"(d), "l"(src), "l"(policy));
+}
+
+__device__ __forceinline__ void cp_async_wait_all()
+{
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
+// Issues the cp.async copies of rows [r0, r0 + rows) of a window (row pointers in rp,
+// NULL = skip; d elements each) into a stage of rows of 32 * EPL floats, and commits
+// them as one group. VEC: 16-byte pieces (d % 4 == 0 and rows 16-byte aligned).
+template <int EPL, bool VEC>
+__device__ __forceinline__ void issue_stage(float *stage, const float *const *rp, int r0, int rows, int d, int lane,
+                                            uint64_t policy)
+{
+    constexpr int ROW = 32 * EPL;
+    const int piece = VEC ? 4 : 1;
+    const int cpr = (d + piece - 1) / piece;  // copies per row
+    if (cpr <= 32) {
+        const int rpi = 32 / cpr;             // rows per pass of the warp
+        const int sub = lane / cpr, col = lane - sub * cpr;
+        if (sub < rpi) {
+            for (int r = sub; r < rows; r += rpi) {
+                const float *src = rp[r0 + r];
+                if (src) {
+                    if (VEC)
+                        cp_async16(stage + r * ROW + col * 4, src + col * 4, policy);
+                    else
+                        cp_async4(stage + r * ROW + col, src + col, policy);
+                }
+            }
         }
     } else {
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-            v[e] = k0 + e < d ? __ldg(row + k0 + e) : 0.0f;
+        for (int r = 0; r < rows; ++r) {
+            const float *src = rp[r0 + r];
+            if (!src)
+                continue;
+            for (int col = lane; col < cpr; col += 32) {
+                if (VEC)
+                    cp_async16(stage + r * ROW + col * 4, src + col * 4, policy);
+                else
+                    cp_async4(stage + r * ROW + col, src + col, policy);
+            }
+        }
     }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
 }
 
-// Lists a finished row: its key and G = the binary64 sum rounded once to binary32.
-template <int EPL>
-__device__ __forceinline__ void list_row(const BwdArgs &a, uint32_t slot, uint32_t key, const double (&s)[EPL],
-                                         int lane)
-{
-    if (lane == 0)
-        a.list[slot] = key;
-    float *gr = a.grad_rows + (int64_t)slot * a.grad_ld + lane * EPL;
-#pragma unroll
-    for (int e = 0; e < EPL; ++e)
-        if (lane * EPL + e < a.d)
-            gr[e] = (float)s[e];
-}
-
-// Window j covers sorted entries [64 j, 64 j + 64). Lane l holds entries l and l + 32.
-// Each block takes 8 consecutive windows per iteration (one per warp) and draws list
-// slots for all of them with one atomic.
+// Blocks take chunks of up to 8 consecutive windows (window j = sorted entries
+// [64 j, 64 j + 64)). Per chunk, the block reads the windows' keys into shared
+// memory, finds each entry's gradient row, and counts the rows whose last entry lies
+// in each window, drawing their list slots with one atomic. Each warp then takes
+// whole windows. Lane l owns elements [l * EPL, l * EPL + EPL) of the rows: EPL
+// independent binary64 chains. The window's gradient rows are copied to shared
+// memory in stages of 32 / EPL rows (4 KB; the next stage's copies are issued before
+// the current one is summed), and the warp walks the window's parts (runs of one
+// row): a part's entries are added in order from +0. A row whose entries all lie in
+// the window is listed with its G; a row that ends here but began earlier is listed
+// too, its G left to bwd_span_kernel (span_slot[j]); a row's part that does not
+// finish it is stored in partials.
 template <int EPL, bool VEC>
-__global__ void __launch_bounds__(kRedThreads) bwd_window_kernel(const BwdArgs a)
+__global__ void __launch_bounds__(kWinWarps * 32) bwd_window_kernel(const BwdArgs a, const int chunk)
 {
-    __shared__ uint32_t warp_cnt[kRedThreads / 32];
-    __shared__ uint32_t block_slot;
+    constexpr int ROW = 32 * EPL;
+    constexpr int SR = kStageFloats / ROW;  // rows per stage, divides 64
+    extern __shared__ __align__(16) float stage_all[];  // [warps][2][kStageFloats]
+    __shared__ const float *rp[kChunk][kWin];
+    __shared__ uint32_t ks[kChunk][kWin + 2];            // the window's keys, then the ones before and after
+    __shared__ uint32_t n_end[kChunk], slot_base[kChunk];
     if (*(volatile uint32_t *)a.hdr)
         return;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    float *stage2 = stage_all + (size_t)warp * 2 * kStageFloats;
+    const uint64_t policy = evict_last_policy();
     const uint32_t sent = a.key_base[a.T];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t *keys = a.keys[0];
     const int32_t *bags = a.bags[0];
     const int64_t windows = (a.n + kWin - 1) / kWin;
     const int64_t row_len = (int64_t)a.T * a.d;
-    for (int64_t jb = (int64_t)blockIdx.x * (kRedThreads / 32); jb < windows; jb += (int64_t)gridDim.x * (kRedThreads / 32)) {
-        const int64_t j = jb + warp;
-        const bool live = j < windows;  // block-uniform loop; a warp past the end only joins the barriers
-        const int64_t w0 = j * kWin;
-        const int cnt = live ? (int)(a.n - w0 < kWin ? a.n - w0 : kWin) : 0;
-        const uint32_t k_lo = lane < cnt ? __ldg(keys + w0 + lane) : sent;
-        const uint32_t k_hi = lane + 32 < cnt ? __ldg(keys + w0 + 32 + lane) : sent;
-        const int32_t g_lo = lane < cnt ? __ldg(bags + w0 + lane) : 0;
-        const int32_t g_hi = lane + 32 < cnt ? __ldg(bags + w0 + 32 + lane) : 0;
-        const uint32_t k_prev = live && j > 0 ? __ldg(keys + w0 - 1) : sent;
-        const uint32_t k_next = live && w0 + kWin < a.n ? __ldg(keys + w0 + kWin) : sent;
-        // neighbours of both entries of the lane
-        const uint32_t up_lo = __shfl_up_sync(0xffffffffu, k_lo, 1), up_hi = __shfl_up_sync(0xffffffffu, k_hi, 1);
-        const uint32_t dn_lo = __shfl_down_sync(0xffffffffu, k_lo, 1), dn_hi = __shfl_down_sync(0xffffffffu, k_hi, 1);
-        const uint32_t lo31 = __shfl_sync(0xffffffffu, k_lo, 31), hi0 = __shfl_sync(0xffffffffu, k_hi, 0);
-        const uint32_t prev_lo = lane == 0 ? k_prev : up_lo, prev_hi = lane == 0 ? lo31 : up_hi;
-        const uint32_t next_lo = lane == 31 ? hi0 : dn_lo, next_hi = lane == 31 ? k_next : dn_hi;
-        (void)prev_lo;
-        (void)prev_hi;
-        // a row is finished here when its last entry is here and it did not start before the window
-        const bool fin_lo = k_lo != sent && k_lo != next_lo && k_lo != k_prev;
-        const bool fin_hi = k_hi != sent && k_hi != next_hi && k_hi != k_prev;
-        const unsigned b_lo = __ballot_sync(0xffffffffu, fin_lo), b_hi = __ballot_sync(0xffffffffu, fin_hi);
-        const uint32_t n_fin = (uint32_t)(__popc(b_lo) + __popc(b_hi));
-        if (lane == 0)
-            warp_cnt[warp] = n_fin;
+    const int k0 = lane * EPL;
+    for (int64_t c0 = (int64_t)blockIdx.x * chunk; c0 < windows; c0 += (int64_t)gridDim.x * chunk) {
+        const int nw = windows - c0 < chunk ? (int)(windows - c0) : chunk;
+        for (int cw = warp; cw < nw; cw += nwarps) {
+            const int64_t j = c0 + cw, w0 = j * kWin;
+            const int cnt = (int)(a.n - w0 < kWin ? a.n - w0 : kWin);
+            const uint32_t k_lo = lane < cnt ? __ldg(keys + w0 + lane) : sent;
+            const uint32_t k_hi = lane + 32 < cnt ? __ldg(keys + w0 + 32 + lane) : sent;
+            const uint32_t k_next = w0 + kWin < a.n ? __ldg(keys + w0 + kWin) : sent;
+            ks[cw][lane] = k_lo;
+            ks[cw][lane + 32] = k_hi;
+            if (lane == 0) {
+                ks[cw][kWin] = j > 0 ? __ldg(keys + w0 - 1) : sent;
+                ks[cw][kWin + 1] = k_next;
+            }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t key = h ? k_hi : k_lo;
+                const float *row = nullptr;
+                if (key != sent) {
+                    const int32_t g = __ldg(bags + w0 + lane + 32 * h);
+                    const int t = (int)div_batch((uint32_t)g, a.div);
+                    row = a.grad + ((int64_t)g - (int64_t)t * a.batch) * row_len + (int64_t)t * a.d;
+                }
+                rp[cw][lane + 32 * h] = row;
+            }
+            const uint32_t dn_lo = __shfl_down_sync(0xffffffffu, k_lo, 1), dn_hi = __shfl_down_sync(0xffffffffu, k_hi, 1);
+            const uint32_t hi0 = __shfl_sync(0xffffffffu, k_hi, 0);
+            const uint32_t next_lo = lane == 31 ? hi0 : dn_lo, next_hi = lane == 31 ? k_next : dn_hi;
+            const bool end_lo = k_lo != sent && k_lo != next_lo, end_hi = k_hi != sent && k_hi != next_hi;
+            const int ends = __popc(__ballot_sync(0xffffffffu, end_lo)) + __popc(__ballot_sync(0xffffffffu, end_hi));
+            if (lane == 0)
+                n_end[cw] = (uint32_t)ends;
+        }
         __syncthreads();
         if (threadIdx.x == 0) {
             uint32_t tot = 0;
-            for (int w = 0; w < kRedThreads / 32; ++w)
-                tot += warp_cnt[w];
-            block_slot = tot ? atomicAdd(a.hdr + 1, tot) : 0u;
+            for (int cw = 0; cw < nw; ++cw) {
+                slot_base[cw] = tot;
+                tot += n_end[cw];
+            }
+            const uint32_t base = tot ? atomicAdd(a.hdr + 1, tot) : 0u;
+            for (int cw = 0; cw < nw; ++cw)
+                slot_base[cw] += base;
         }
         __syncthreads();
-        uint32_t slot = block_slot;
-        for (int w = 0; w < warp; ++w)
-            slot += warp_cnt[w];
-        __syncthreads();  // warp_cnt and block_slot are rewritten next iteration
-        if (!live)
-            continue;
-
-        double acc[EPL];
-#pragma unroll
-        for (int e = 0; e < EPL; ++e)
-            acc[e] = 0.0;
-        bool from_before = true;  // the current part began at the window's first entry
-        constexpr int U = EPL <= 4 ? 8 : (EPL <= 8 ? 4 : 2);
-        for (int i0 = 0; i0 < cnt; i0 += U) {
-            // gather U entries and issue their gradient loads before any add
-            float gv[U][EPL];
-            uint32_t kk[U];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = i0 + u;
-                const uint32_t ksrc = i < 32 ? k_lo : k_hi;
-                const int32_t gsrc = i < 32 ? g_lo : g_hi;
-                kk[u] = __shfl_sync(0xffffffffu, ksrc, i & 31);
-                const int32_t g = __shfl_sync(0xffffffffu, gsrc, i & 31);
-                const bool ok = i < cnt && kk[u] != sent;
-                const int t = (int)div_batch((uint32_t)g, a.div);
-                const int64_t b = (int64_t)g - (int64_t)t * a.batch;
-                const float *row = a.grad + b * row_len + (int64_t)t * a.d;
-                if (ok)
-                    load_elems<EPL, VEC>(row, lane, a.d, gv[u]);
-                else {
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e)
-                        gv[u][e] = 0.0f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int i = i0 + u;
-                if (i >= cnt || kk[u] == sent)
-                    break;  // uniform: the sentinel entries come last
-#pragma unroll
-                for (int e = 0; e < EPL; ++e)
-                    acc[e] = acc[e] + (double)gv[u][e];
-                const uint32_t nsrc = i < 32 ? next_lo : next_hi;
-                const uint32_t knext = __shfl_sync(0xffffffffu, nsrc, i & 31);
-                const bool part_end = knext != kk[u] || i == cnt - 1;
-                if (!part_end)
-                    continue;
-                const bool began_before = from_before && kk[u] == k_prev;
-                const bool goes_on = knext == kk[u];  // only at the window's last entry
-                if (!began_before && !goes_on) {
-                    list_row<EPL>(a, slot, kk[u], acc, lane);
-                    ++slot;
-                } else {
-                    // the row's part: slot 1 = the part of the window where it starts,
-                    // slot 0 = a part that began in an earlier window
-                    const int which = began_before ? 0 : 1;
-                    double *pp = a.partials + ((j * 2 + which) * (int64_t)a.d) + lane * EPL;
-#pragma unroll
-                    for (int e = 0; e < EPL; ++e)
-                        if (lane * EPL + e < a.d)
-                            pp[e] = acc[e];
-                }
-#pragma unroll
-                for (int e = 0; e < EPL; ++e)
-                    acc[e] = 0.0;
-                from_before = false;
-            }
+        // this warp's stages: windows warp, warp + nwarps, ... of the chunk, 64 / SR each
+        auto win_cnt = [&](int cw) { return (int)(a.n - (c0 + cw) * kWin < kWin ? a.n - (c0 + cw) * kWin : kWin); };
+        int buf = 0;
+        if (warp < nw) {
+            const int c = win_cnt(warp);
+            issue_stage<EPL, VEC>(stage2, rp[warp], 0, c < SR ? c : SR, a.d, lane, policy);
         }
+        for (int cw = warp; cw < nw; cw += nwarps) {
+            const int64_t j = c0 + cw;
+            const int cnt = win_cnt(cw);
+            const uint32_t k_lo = ks[cw][lane], k_hi = ks[cw][lane + 32];
+            const uint32_t k_prev = ks[cw][kWin], k_next = ks[cw][kWin + 1];
+            const uint32_t nx_lo = ks[cw][lane + 1];
+            const uint32_t nx_hi = lane == 31 ? k_next : ks[cw][lane + 33];
+            // valid entries form a prefix (invalid ones sort last); part ends as a mask
+            const unsigned v_lo = __ballot_sync(0xffffffffu, k_lo != sent), v_hi = __ballot_sync(0xffffffffu, k_hi != sent);
+            const int nv = __popc(v_lo) + __popc(v_hi);
+            uint64_t ends = (uint64_t)__ballot_sync(0xffffffffu, k_lo != sent && k_lo != nx_lo) |
+                            ((uint64_t)__ballot_sync(0xffffffffu, k_hi != sent && k_hi != nx_hi) << 32);
+            if (nv == cnt && nv > 0)
+                ends |= 1ull << (nv - 1);  // the window's last entry ends a part even if its row goes on
+            uint32_t slot = slot_base[cw], span_slot = kNoSpan;
+            double acc[EPL];
+#pragma unroll
+            for (int e = 0; e < EPL; ++e)
+                acc[e] = 0.0;
+            int i = 0;  // next entry to add
+            bool first_part = true;
+            for (int s0 = 0; s0 < cnt; s0 += SR, buf ^= 1) {
+                // the stage after this one (this window's next, or the warp's next window's first)
+                const int ns0 = s0 + SR;
+                const bool more_here = ns0 < cnt;
+                const int ncw = cw + nwarps;
+                if (more_here) {
+                    issue_stage<EPL, VEC>(stage2 + (buf ^ 1) * kStageFloats, rp[cw], ns0,
+                                          cnt - ns0 < SR ? cnt - ns0 : SR, a.d, lane, policy);
+                    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+                } else if (ncw < nw) {
+                    const int c = win_cnt(ncw);
+                    issue_stage<EPL, VEC>(stage2 + (buf ^ 1) * kStageFloats, rp[ncw], 0, c < SR ? c : SR, a.d, lane,
+                                          policy);
+                    asm volatile("cp.async.wait_group 1;\n" ::: "memory");
+                } else {
+                    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
+                }
+                __syncwarp();
+                const float *stage = stage2 + buf * kStageFloats + k0;
+                const int s1 = s0 + SR < nv ? s0 + SR : nv;  // entries of this stage to add
+                while (i < s1) {
+                    const int e_end = ends ? __ffsll((long long)ends) - 1 : kWin;
+                    const int stop = e_end < s1 ? e_end + 1 : s1;
+                    for (; i < stop; ++i) {
+                        const float *v = stage + (i - s0) * ROW;
+                        if constexpr (EPL >= 4) {
+#pragma unroll
+                            for (int e = 0; e < EPL; e += 4) {
+                                const float4 q = *reinterpret_cast<const float4 *>(v + e);
+                                acc[e] = acc[e] + (double)q.x;
+                                acc[e + 1] = acc[e + 1] + (double)q.y;
+                                acc[e + 2] = acc[e + 2] + (double)q.z;
+                                acc[e + 3] = acc[e + 3] + (double)q.w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < EPL; ++e)
+                                acc[e] = acc[e] + (double)v[e];
+                        }
+                    }
+                    if (stop != e_end + 1)
+                        break;  // the part goes on into the next stage
+                    ends &= ends - 1;
+                    const uint32_t key = ks[cw][e_end];
+                    const bool began_before = first_part && key == k_prev;
+                    const bool goes_on = e_end == kWin - 1 && key == k_next;
+                    if (!began_before && !goes_on) {
+                        if (lane == 0)
+                            a.list[slot] = key;
+                        float *gr = a.grad_rows + (int64_t)slot * a.grad_ld + k0;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e)
+                            if (k0 + e < a.d)
+                                __stcs(gr + e, (float)acc[e]);
+                        ++slot;
+                    } else {
+                        // slot 1 = the part of the window where the row starts,
+                        // slot 0 = a part of a row that began in an earlier window
+                        const int which = began_before ? 0 : 1;
+                        double *pp = a.partials + (j * 2 + which) * (int64_t)a.d + k0;
+#pragma unroll
+                        for (int e = 0; e < EPL; ++e)
+                            if (k0 + e < a.d)
+                                __stcs(pp + e, acc[e]);
+                        if (began_before && !goes_on) {
+                            if (lane == 0)
+                                a.list[slot] = key;
+                            span_slot = slot++;
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < EPL; ++e)
+                        acc[e] = 0.0;
+                    first_part = false;
+                }
+                __syncwarp();  // this stage is refilled two stages on
+            }
+            if (lane == 0)
+                a.span_slot[j] = span_slot;
+        }
+        __syncthreads();  // rp, ks, n_end and slot_base are rewritten for the next chunk
     }
 }
 
-// Rows spanning windows: found at the window where they end (their first entry of
-// the window continues the previous window's last row, and they end inside it).
-template <int EPL>
-__global__ void __launch_bounds__(kRedThreads) bwd_span_kernel(const BwdArgs a)
+// G of the rows that span windows, listed by bwd_window_kernel at the window where
+// they end: the parts in window order, summed in binary64. One warp per (window,
+// 32-element slice of the row), one element per lane; the parts of 32 windows at a
+// time are copied to shared memory first (cp.async), so their loads are all in flight.
+constexpr int kSpanWarps = 4;
+constexpr int kSpanAhead = 32;
+
+__device__ __forceinline__ void cp_async8(void *dst, const void *src)
 {
+    const unsigned d = (unsigned)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(d), "l"(src));
+}
+
+__global__ void __launch_bounds__(kSpanWarps * 32) bwd_span_kernel(const BwdArgs a)
+{
+    __shared__ double ahead[kSpanWarps][kSpanAhead][32];
     if (*(volatile uint32_t *)a.hdr)
         return;
-    const uint32_t sent = a.key_base[a.T];
-    const int lane = threadIdx.x & 31;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const uint32_t *keys = a.keys[0];
     const int64_t windows = (a.n + kWin - 1) / kWin;
+    const int slices = (a.d + 31) / 32;
+    const int64_t items = windows * slices;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    for (int64_t j = 1 + warp0; j < windows; j += warps) {
+    for (int64_t it = warp0; it < items; it += warps) {
+        const int64_t j = it / slices;
+        const int slice = (int)(it - j * slices);
+        const uint32_t slot = __ldg(a.span_slot + j);
+        if (slot == kNoSpan)
+            continue;
+        // the row's first entry: keys[64 j - 1] == keys[64 j] == k0; gallop back, then bisect
         const int64_t w0 = j * kWin;
         const uint32_t k0 = __ldg(keys + w0);
-        if (k0 == sent || __ldg(keys + w0 - 1) != k0)
-            continue;
-        const int cnt = (int)(a.n - w0 < kWin ? a.n - w0 : kWin);
-        const bool other_lo = lane < cnt && __ldg(keys + w0 + lane) != k0;
-        const bool other_hi = lane + 32 < cnt && __ldg(keys + w0 + 32 + lane) != k0;
-        const bool ends_inside = __any_sync(0xffffffffu, other_lo || other_hi);
-        if (!ends_inside && cnt == kWin && w0 + kWin < a.n && __ldg(keys + w0 + kWin) == k0)
-            continue;  // the row goes on into the next window
-        // first entry of the row: lower bound of k0 in [0, w0)
-        int64_t lo = 0, hi = w0;
-        while (lo < hi) {
+        int64_t hi = w0 - 1, step = kWin, lo = hi - step;
+        while (lo >= 0 && __ldg(keys + lo) == k0) {
+            hi = lo;
+            step *= 2;
+            lo = hi - step;
+        }
+        if (lo < -1)
+            lo = -1;
+        while (hi - lo > 1) {  // keys[lo] < k0 (or lo == -1), keys[hi] == k0
             const int64_t mid = (lo + hi) >> 1;
-            if (__ldg(keys + mid) < k0)
-                lo = mid + 1;
-            else
+            if (__ldg(keys + mid) == k0)
                 hi = mid;
+            else
+                lo = mid;
         }
-        const int64_t j0 = lo / kWin;
-        double s[EPL];
-        {
-            const double *p = a.partials + (j0 * 2 + 1) * (int64_t)a.d + lane * EPL;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e)
-                s[e] = lane * EPL + e < a.d ? p[e] : 0.0;
+        const int64_t j0 = hi / kWin;
+        const int k = slice * 32 + lane;
+        const bool ok = k < a.d;
+        double s = ok ? a.partials[(j0 * 2 + 1) * (int64_t)a.d + k] : 0.0;
+        for (int64_t jb = j0 + 1; jb <= j; jb += kSpanAhead) {
+            const int m = j - jb + 1 < kSpanAhead ? (int)(j - jb + 1) : kSpanAhead;
+            if (ok)
+                for (int u = 0; u < m; ++u)
+                    cp_async8(&ahead[warp][u][lane], a.partials + ((jb + u) * 2) * (int64_t)a.d + k);
+            cp_async_wait_all();
+            for (int u = 0; u < m; ++u)
+                s = s + ahead[warp][u][lane];
         }
-        for (int64_t jj = j0 + 1; jj <= j; ++jj) {
-            const double *p = a.partials + (jj * 2) * (int64_t)a.d + lane * EPL;
-#pragma unroll
-            for (int e = 0; e < EPL; ++e)
-                s[e] = s[e] + (lane * EPL + e < a.d ? p[e] : 0.0);
-        }
-        uint32_t slot = 0;
-        if (lane == 0)
-            slot = atomicAdd(a.hdr + 1, 1u);
-        slot = __shfl_sync(0xffffffffu, slot, 0);
-        list_row<EPL>(a, slot, k0, s, lane);
+        if (ok)
+            a.grad_rows[(int64_t)slot * a.grad_ld + k] = (float)s;
     }
 }
 
 template <int EPL>
-cudaError_t launch_reduce(const BwdArgs &a, int num_sms, cudaStream_t stream)
+cudaError_t launch_window(const BwdArgs &a, int num_sms, cudaStream_t stream)
 {
     const int64_t windows = (a.n + kWin - 1) / kWin;
-    const int64_t blocks = (windows + kRedThreads / 32 - 1) / (kRedThreads / 32);
-    const int64_t cap = (int64_t)num_sms * 8;
-    const unsigned grid = (unsigned)(blocks < cap ? blocks : cap);
-    const bool vec = EPL >= 4 && a.d % 4 == 0 && ((int64_t)a.T * a.d) % 4 == 0 &&
-                     (reinterpret_cast<uintptr_t>(a.grad) & 15) == 0;
-    if (vec) {
-        if constexpr (EPL >= 4)
-            bwd_window_kernel<EPL, true><<<grid, kRedThreads, 0, stream>>>(a);
-    } else {
-        bwd_window_kernel<EPL, false><<<grid, kRedThreads, 0, stream>>>(a);
+    // chunks of up to 8 windows (about 24 warps per SM: 8 KB of stages per warp),
+    // smaller when there are too few windows to fill the GPU
+    int chunk = kChunk, wpb = kWinWarps;
+    int64_t blocks_wanted = 0;
+    for (;; chunk >>= 1) {
+        wpb = chunk < kWinWarps ? chunk : kWinWarps;
+        blocks_wanted = (int64_t)num_sms * (24 / wpb);
+        if (chunk == 1 || (windows + chunk - 1) / chunk >= blocks_wanted)
+            break;
     }
-    cudaError_t e = cudaGetLastError();
+    const int64_t chunks = (windows + chunk - 1) / chunk;
+    const unsigned grid = (unsigned)(chunks < blocks_wanted ? chunks : blocks_wanted);
+    const size_t smem = (size_t)wpb * 2 * kStageFloats * sizeof(float);
+    const bool vec = a.d % 4 == 0 && ((int64_t)a.T * a.d) % 4 == 0 && (reinterpret_cast<uintptr_t>(a.grad) & 15) == 0;
+    cudaError_t e;
+    if (vec) {
+        e = cudaFuncSetAttribute(bwd_window_kernel<EPL, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            bwd_window_kernel<EPL, true><<<grid, wpb * 32, smem, stream>>>(a, chunk);
+    } else {
+        e = cudaFuncSetAttribute(bwd_window_kernel<EPL, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e == cudaSuccess)
+            bwd_window_kernel<EPL, false><<<grid, wpb * 32, smem, stream>>>(a, chunk);
+    }
     if (e != cudaSuccess)
         return e;
-    if (windows > 1)
-        bwd_span_kernel<EPL><<<grid, kRedThreads, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_reduce(const BwdArgs &a, int num_sms, cudaStream_t stream)
+{
+    int epl = 1;
+    while (epl * 32 < a.d)
+        epl <<= 1;
+    cudaError_t e;
+    switch (epl) {
+    case 1: e = launch_window<1>(a, num_sms, stream); break;
+    case 2: e = launch_window<2>(a, num_sms, stream); break;
+    case 4: e = launch_window<4>(a, num_sms, stream); break;
+    case 8: e = launch_window<8>(a, num_sms, stream); break;
+    case 16: e = launch_window<16>(a, num_sms, stream); break;
+    case 32: e = launch_window<32>(a, num_sms, stream); break;
+    default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess)
+        return e;
+    const int64_t windows = (a.n + kWin - 1) / kWin;
+    if (windows > 1) {
+        const int64_t items = windows * ((a.d + 31) / 32);
+        const int64_t need = (items + kSpanWarps - 1) / kSpanWarps;
+        const int64_t cap2 = (int64_t)num_sms * 16;
+        bwd_span_kernel<<<(unsigned)(need < cap2 ? need : cap2), kSpanWarps * 32, 0, stream>>>(a);
+    }
     return cudaGetLastError();
 }
 
@@ -502,6 +660,7 @@ BwdLayout bwd_layout(int64_t n, int d)
     L.hist = take((size_t)kDigits * (size_t)L.tiles * 4);
     L.totals = take((size_t)kDigits * 4);
     L.partials = take((size_t)L.windows * 2 * (size_t)d * 8);
+    L.span_slot = take((size_t)L.windows * 4);
     L.list = take((size_t)n * 4);
     L.grad_rows = take((size_t)n * (size_t)L.grad_ld * 4);
     L.total = off;
@@ -513,9 +672,14 @@ cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream)
 {
     const int64_t G = (int64_t)a.T * a.batch;
     {
-        const int64_t need = (G + 255) / 256;
+        const bool warp_per_bag = a.n >= 8 * G;
+        const int64_t need = warp_per_bag ? (G * 32 + 255) / 256 : (G + 255) / 256;
         const int64_t cap = (int64_t)num_sms * 16;
-        bwd_keys_kernel<<<(unsigned)(need < cap ? need : cap), 256, 0, stream>>>(a);
+        const unsigned grid = (unsigned)(need < cap ? need : cap);
+        if (warp_per_bag)
+            bwd_keys_kernel<true><<<grid, 256, 0, stream>>>(a);
+        else
+            bwd_keys_kernel<false><<<grid, 256, 0, stream>>>(a);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess)
             return e;
@@ -541,18 +705,7 @@ cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream)
         a.bags[0] = a.bags[1];
         a.bags[1] = tb;
     }
-    int epl = 1;
-    while (epl * 32 < a.d)
-        epl <<= 1;
-    switch (epl) {
-    case 1: return launch_reduce<1>(a, num_sms, stream);
-    case 2: return launch_reduce<2>(a, num_sms, stream);
-    case 4: return launch_reduce<4>(a, num_sms, stream);
-    case 8: return launch_reduce<8>(a, num_sms, stream);
-    case 16: return launch_reduce<16>(a, num_sms, stream);
-    case 32: return launch_reduce<32>(a, num_sms, stream);
-    default: return cudaErrorInvalidValue;
-    }
+    return launch_reduce(a, num_sms, stream);
 }
 
 } // namespace dq

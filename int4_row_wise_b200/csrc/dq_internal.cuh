@@ -109,6 +109,7 @@ struct BwdArgs {
     uint32_t *hist;            // [256][tiles]
     uint32_t *totals;          // [256]
     double *partials;          // [windows][2][d]
+    uint32_t *span_slot;       // [windows] list slot of the spanning row ending there
     uint32_t *list;            // [entries]
     float *grad_rows;          // [entries][grad_ld]
     int64_t grad_ld;
@@ -117,7 +118,7 @@ struct BwdArgs {
 
 // Byte offsets of the pieces of the backward's workspace (each 256-byte aligned).
 struct BwdLayout {
-    size_t hdr, keys0, keys1, bags0, bags1, hist, totals, partials, list, grad_rows, total;
+    size_t hdr, keys0, keys1, bags0, bags1, hist, totals, partials, span_slot, list, grad_rows, total;
     int64_t tiles, windows, grad_ld;
 };
 BwdLayout bwd_layout(int64_t n, int d);
