@@ -476,6 +476,85 @@ def run_lookup_only(args, wl: W.Workload) -> None:
         "gpu_launches": args.steps}), flush=True)
 
 
+def _touched_rows(wl: W.Workload, idx: np.ndarray, off: np.ndarray) -> int:
+    """Distinct (table, row) pairs of one lookup batch: the rows its backward updates."""
+    B = wl.batch
+    return int(sum(np.unique(idx[off[t * B]:off[(t + 1) * B]]).size for t in range(wl.n_tables)))
+
+
+def run_bwd(args, wl: W.Workload) -> None:
+    """Times the training step after the lookup (dq_embbag_int4_bwd_sgd): the bag
+    backward, the SGD step on binary32 masters of the workload's table sizes and the
+    re-quantization of the touched rows, over 4 distinct lookup batches, each with its
+    own output gradient. Masters and gradients are seeded normal draws on the device."""
+    import torch
+    import int4_row_wise_b200 as dq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dq.load()
+    d = wl.d
+    cld = dq._codes_ld(d)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    tables = []
+    for n in wl.rows:
+        m = torch.randn((n, d), generator=gen, device=dev)
+        c, sb, _, _ = dq.quantize_rows(m, with_loss=False)
+        tables.append(dq.MasterTable(m, c, sb))
+    n_batches = 4
+    bh = [W.lookup_batch(wl, batch_id=i) for i in range(n_batches)]
+    bd = [(torch.from_numpy(i).to(dev), torch.from_numpy(o).to(dev)) for i, o in bh]
+    grads = [torch.randn((wl.batch, wl.n_tables * d), generator=gen, device=dev) * 1e-2 for _ in range(n_batches)]
+    touched = [_touched_rows(wl, i, o) for i, o in bh]
+    n_ids = [int(i.size) for i, _ in bh]
+    ws = torch.empty(max(dq.dq_embbag_int4_bwd_workspace_bytes(d, max(n_ids)), 256), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    lr = 0.05
+
+    def call(k):
+        i, o = bd[k % n_batches]
+        dq.dq_embbag_int4_bwd_sgd(tables, d, i, o, wl.batch, n_ids[k % n_batches], grads[k % n_batches], lr,
+                                  dq.DQ_MODE_GREEDY, ws, ws.numel(), None, stream)
+
+    for k in range(args.warmup):
+        call(k)
+    torch.cuda.synchronize(dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(0) as clocks:
+        for k in range(args.steps):
+            flush.zero_()
+            evs[k][0].record(stream)
+            call(k)
+            evs[k][1].record(stream)
+        torch.cuda.synchronize(dev)
+    clk = clocks.summary()
+    ms = [a.elapsed_time(b) for a, b in evs]
+    tot_ms = sum(ms)
+    ids = sum(n_ids[k % n_batches] for k in range(args.steps))
+    rows = sum(touched[k % n_batches] for k in range(args.steps))
+    # the re-quantization's FP32 work (3370 d flops per touched row) against the FP32 peak,
+    # over the whole call: a lower bound for requant_rows_kernel, which is most of it
+    flops = rows * EVALS_PER_ROW * 10 * d
+    peak = 2 * FP32_LANES_PER_SM * torch.cuda.get_device_properties(dev).multi_processor_count * 1965e6 / 1e12
+    tflops = flops / (tot_ms / 1e3) / 1e12
+    bits = max(1, int(sum(wl.rows)).bit_length())
+    launches = 1 + 3 * ((bits + 7) // 8) + 3  # keys, sort passes, window, span, re-quantization
+    print(json.dumps({
+        "metric": "INT4 bag backward + SGD on binary32 masters + greedy re-quantization of touched rows: ids/s",
+        "value": ids / (tot_ms / 1e3), "unit": "ids/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_ms / len(ms), "higher_is_better": True, "dtype": "f32 (f64 gradient sums)",
+        "data": "synthetic",
+        "config": {"workload": _workload_desc(wl), "ids_per_call": int(np.mean(n_ids)),
+                   "touched_rows_per_call": int(np.mean(touched)), "lr": lr,
+                   "masters": "seeded normal draws of the workload's table sizes",
+                   "l2": "256 MB flush written before every call"},
+        "touched_rows_per_s": rows / (tot_ms / 1e3),
+        "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s", "frac": tflops / peak,
+                     "over": "the whole call (re-quantization flops only)"},
+        "clocks": clk, "gpu_launches": launches * args.steps}), flush=True)
+
+
 def _measured_hbm() -> float:
     try:
         return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
@@ -575,6 +654,8 @@ def main(argv=None) -> None:
     ap.add_argument("--lookup-only", action="store_true",
                     help="time only the lookup, over random packed tables of the workload's sizes")
     ap.add_argument("--streams", type=int, default=4, help="streams the per-table quantize launches spread over")
+    ap.add_argument("--bwd", action="store_true",
+                    help="time the bag backward + SGD + re-quantization over masters of the workload's sizes")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -583,6 +664,8 @@ def main(argv=None) -> None:
         run_reference(args, wl)
     elif args.lookup_only:
         run_lookup_only(args, wl)
+    elif args.bwd:
+        run_bwd(args, wl)
     else:
         run_gpu(args, wl)
 

@@ -65,7 +65,7 @@ def lib():
             L.oracle_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp]
             L.oracle_row_l2_error.restype = ctypes.c_double
             L.oracle_embbag_bwd_sgd.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, vp, vp, i32, i64, vp,
-                                                ctypes.c_float, i32]
+                                                ctypes.c_float, i32, vp, i64]
             L.oracle_embbag_bwd_sgd.restype = i64
             L.oracle_embbag.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, i32]
             L.oracle_embbag.restype = i64
@@ -190,11 +190,12 @@ BAD_OFFSETS = -2
 
 
 def embbag_bwd_sgd(masters, codes, scale_bias, d: int, indices: np.ndarray, offsets: np.ndarray,
-                   batch: int, grad: np.ndarray, lr: float, mode: int = GREEDY) -> int:
+                   batch: int, grad: np.ndarray, lr: float, mode: int = GREEDY, sample_keys=None) -> int:
     """Bag backward, SGD step on the binary32 masters and re-quantization of the touched
     rows, all in place. masters: list of float32 [n, ld]; codes: list of uint8 [n, cld];
-    scale_bias: list of uint16 [n, 2]; grad: float32 [batch, T*d]. Returns the number of
-    invalid ids, or BAD_OFFSETS when the offsets are not a CSR array (nothing changed)."""
+    scale_bias: list of uint16 [n, 2]; grad: float32 [batch, T*d]. sample_keys (global
+    keys = rows of the tables before t + id): update only those rows. Returns the number
+    of invalid ids, or BAD_OFFSETS when the offsets are not a CSR array (nothing changed)."""
     T = len(masters)
     for w, c, sb in zip(masters, codes, scale_bias):
         assert w.dtype == np.float32 and w.flags["C_CONTIGUOUS"]
@@ -210,8 +211,10 @@ def embbag_bwd_sgd(masters, codes, scale_bias, d: int, indices: np.ndarray, offs
     idx = np.ascontiguousarray(indices, dtype=np.int32)
     off = np.ascontiguousarray(offsets, dtype=np.int32)
     g = np.ascontiguousarray(grad, dtype=np.float32)
+    sk = None if sample_keys is None else np.ascontiguousarray(np.unique(sample_keys), dtype=np.uint32)
     r = lib().oracle_embbag_bwd_sgd(ptrs(masters), _p(wld), ptrs(codes), _p(cld), ptrs(scale_bias), _p(nrows),
-                                    T, d, _p(idx), _p(off), batch, int(idx.size), _p(g), np.float32(lr), mode)
+                                    T, d, _p(idx), _p(off), batch, int(idx.size), _p(g), np.float32(lr), mode,
+                                    None if sk is None else _p(sk), 0 if sk is None else int(sk.size))
     if r == -1:
         raise ValueError("oracle_embbag_bwd_sgd: bad arguments")
     return int(r)

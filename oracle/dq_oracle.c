@@ -510,15 +510,30 @@ static int entry_cmp(const void *pa, const void *pb)
     return a->pos < b->pos ? -1 : (a->pos > b->pos ? 1 : 0);
 }
 
+/* key in the ascending array sample[0..n)? */
+static int in_sample(const uint32_t *sample, int64_t n, uint32_t key)
+{
+    int64_t lo = 0, hi = n;
+    while (lo < hi) {
+        int64_t mid = lo + (hi - lo) / 2;
+        if (sample[mid] < key)
+            lo = mid + 1;
+        else
+            hi = mid;
+    }
+    return lo < n && sample[lo] == key;
+}
+
 /* Steps a-e of the bag backward on T tables sharing d: masters W[t] (row stride
  * w_ld[t]) and packed tables codes[t]/scale_bias[t] (code row stride codes_ld[t]),
- * n_rows[t] rows each; grad is [B][T*d]. Returns the number of invalid ids, -2 if the
+ * n_rows[t] rows each; grad is [B][T*d]. With sample_keys (ascending global keys), steps
+ * c-e are applied to those rows only. Returns the number of invalid ids, -2 if the
  * offsets are not a CSR array (nothing changed), -1 on bad arguments. */
 int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *const *codes,
                               const int64_t *codes_ld, uint16_t *const *scale_bias,
                               const int64_t *n_rows, int32_t T, int32_t d, const int32_t *indices,
                               const int32_t *offsets, int32_t B, int64_t n_indices, const float *grad,
-                              float lr, int32_t mode)
+                              float lr, int32_t mode, const uint32_t *sample_keys, int64_t n_sample)
 {
     if (T < 1 || d < 1 || d > ORACLE_MAX_D || B < 0 || n_indices < 0)
         return -1;
@@ -560,6 +575,10 @@ int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *con
         int64_t s1 = s0;
         while (s1 < ne && e[s1].key == e[s0].key)
             s1++;
+        if (sample_keys && !in_sample(sample_keys, n_sample, e[s0].key)) {
+            s0 = s1;  /* steps c-e only for the sampled rows (the windows still count every entry) */
+            continue;
+        }
         int t = 0;
         while (t + 1 < T && (int64_t)e[s0].key >= row_base[t + 1])
             t++;

@@ -98,3 +98,47 @@ def test_lookup_full_call(cuda_device, name):
         bag_tolerance_check(got, ref, mag)
         if wl.pooling == (1, 1):
             assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
+
+
+def test_bwd_full_kaggle_call(cuda_device):
+    """The bag backward + SGD + re-quantization on the Kaggle-shaped workload's own
+    tables (all 26, 12.1M rows) and its full lookup batch, as bench.py --bwd launches
+    it. Sampled rows (the hottest ones, which span many windows, and random touched
+    ones) against the oracle bit for bit; sampled untouched rows unchanged. (Training
+    step of "Deep Quantized Recommendation Model (DQRM)", repository page.)"""
+    wl = W.workload("kaggle")
+    d, B, T = wl.d, wl.batch, wl.n_tables
+    cld = dq._codes_ld(d)
+    rng = np.random.default_rng(31)
+    masters = [np.ascontiguousarray(W.table_rows(wl, t)) for t in range(T)]
+    codes = [rng.integers(0, 256, (n, cld), dtype=np.uint8) for n in wl.rows]
+    sbs = [rng.integers(0, 1 << 16, (n, 2), dtype=np.uint16) for n in wl.rows]
+    idx, off = W.lookup_batch(wl, 0)
+    grad = rng.standard_normal((B, T * d)).astype(np.float32)
+    lr = 0.05
+    tabs = [dq.MasterTable(to_dev(m), to_dev(c), to_dev(s.view(np.int16))) for m, c, s in zip(masters, codes, sbs)]
+    dq.embbag_bwd_sgd(tabs, d, to_dev(idx), to_dev(off), B, to_dev(grad), lr)
+    torch.cuda.synchronize()
+    # rows touched, with their entry counts
+    base = np.concatenate([[0], np.cumsum(wl.rows)]).astype(np.int64)
+    t_of = np.repeat(np.arange(T), [off[(t + 1) * B] - off[t * B] for t in range(T)])
+    keys, counts = np.unique(base[t_of] + idx.astype(np.int64), return_counts=True)
+    hot = keys[np.argsort(-counts)[:20]]
+    sample = np.unique(np.concatenate([hot, rng.choice(keys, 2000, replace=False)]))
+    assert counts.max() > 64  # some rows span windows of the sorted entries
+    oracle.embbag_bwd_sgd(masters, codes, sbs, d, idx, off, B, grad, lr, sample_keys=sample)
+    for key in sample:
+        t = int(np.searchsorted(base, key, side="right") - 1)
+        r = int(key - base[t])
+        assert np.array_equal(tabs[t].master[r].cpu().numpy().view(np.uint32), masters[t][r].view(np.uint32)), key
+        assert np.array_equal(tabs[t].codes[r].cpu().numpy(), codes[t][r]), key
+        assert np.array_equal(tabs[t].scale_bias[r].cpu().numpy().view(np.uint16), sbs[t][r]), key
+    # untouched rows keep their values (the host arrays still hold the inputs there)
+    for t in range(0, T, 5):
+        n = wl.rows[t]
+        rows = rng.choice(n, min(n, 500), replace=False)
+        mine = keys[(keys >= base[t]) & (keys < base[t + 1])] - base[t]
+        rows = np.setdiff1d(rows, mine)
+        rt = torch.from_numpy(rows).cuda()
+        assert np.array_equal(tabs[t].master[rt].cpu().numpy(), masters[t][rows])
+        assert np.array_equal(tabs[t].codes[rt].cpu().numpy(), codes[t][rows])

@@ -172,3 +172,23 @@ def test_min_max_mode_requantizes_with_min_max():
     c, sb, _, _ = oracle.quantize_rows(np.ascontiguousarray(W[0][[2, 5]]), mode=oracle.MINMAX)
     assert np.array_equal(C[0][[2, 5]], c) and np.array_equal(S[0][[2, 5]], sb)
     assert not C[0][[0, 1, 3, 4]].any()
+
+
+def test_sample_updates_exactly_the_sampled_rows():
+    # a sample restricts steps c-e to its rows; each sampled row gets what the full
+    # call gives it (the windows still count every entry)
+    T, B, n, d = 2, 60, 40, 4
+    W, C, S = _tables(T, n, d, 21)
+    idx, off = _bags(T, B, n, 1, 9, 22)
+    g = np.random.default_rng(23).standard_normal((B, T * d)).astype(np.float32)
+    full = ([w.copy() for w in W], [c.copy() for c in C], [s.copy() for s in S])
+    oracle.embbag_bwd_sgd(*full, d, idx, off, B, g, 0.1)
+    part = ([w.copy() for w in W], [c.copy() for c in C], [s.copy() for s in S])
+    keys = np.array([0, 7, n + 3, n + 39], np.uint32)  # rows 0, 7 of table 0; 3, 39 of table 1
+    oracle.embbag_bwd_sgd(*part, d, idx, off, B, g, 0.1, sample_keys=keys)
+    picked = {(0, 0), (0, 7), (1, 3), (1, 39)}
+    for t in range(T):
+        for r in range(n):
+            src = full if (t, r) in picked else (W, C, S)
+            for k in range(3):
+                assert np.array_equal(part[k][t][r], src[k][t][r]), (t, r, k)
