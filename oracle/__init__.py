@@ -42,7 +42,7 @@ def build(force: bool = False) -> str:
 
 class _Table(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scale_bias", ctypes.c_void_p),
-                ("n_rows", ctypes.c_int64), ("codes_ld", ctypes.c_int64)]
+                ("n_rows", ctypes.c_int64), ("codes_ld", ctypes.c_int64), ("codebook", ctypes.c_void_p)]
 
 
 def lib():
@@ -68,6 +68,10 @@ def lib():
                                                 ctypes.c_float, i32, vp, i64]
             L.oracle_embbag_bwd_sgd.restype = i64
             L.oracle_embbag.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, i32]
+            L.oracle_quantize_rows_kmeans.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, i32, i32]
+            L.oracle_quantize_rows_kmeans.restype = i32
+            L.oracle_dequantize_rows_kmeans.argtypes = [vp, i64, vp, i64, i32, vp, i64]
+            L.oracle_dequantize_rows_kmeans.restype = i32
             L.oracle_embbag.restype = i64
             _lib = L
     return _lib
@@ -162,8 +166,9 @@ def row_l2_error(x: np.ndarray, codes: np.ndarray, scale_bias: np.ndarray):
 
 
 def embbag(tables, d: int, indices: np.ndarray, offsets: np.ndarray, batch: int,
-           with_abs_sum: bool = False, nthreads: int = 0):
-    """tables: list of (codes uint8 [n, ld], scale_bias uint16 [n, 2]).
+           with_abs_sum: bool = False, nthreads: int = 0, codebook: bool = False):
+    """tables: list of (codes uint8 [n, ld], scale_bias uint16 [n, 2]), or with codebook=True
+    list of (codes uint8 [n, ld], codebook uint16 [n, 16]).
 
     Returns (out float32 [batch, T*d], abs_sum float64 or None, skipped count)."""
     keep = []
@@ -172,7 +177,10 @@ def embbag(tables, d: int, indices: np.ndarray, offsets: np.ndarray, batch: int,
         codes = np.ascontiguousarray(codes, dtype=np.uint8)
         sb = np.ascontiguousarray(sb, dtype=np.uint16)
         keep += [codes, sb]
-        arr[t] = _Table(codes.ctypes.data, sb.ctypes.data, codes.shape[0], codes.shape[1])
+        if codebook:
+            arr[t] = _Table(codes.ctypes.data, None, codes.shape[0], codes.shape[1], sb.ctypes.data)
+        else:
+            arr[t] = _Table(codes.ctypes.data, sb.ctypes.data, codes.shape[0], codes.shape[1], None)
     idx = np.ascontiguousarray(indices, dtype=np.int32)
     off = np.ascontiguousarray(offsets, dtype=np.int32)
     T = len(tables)
@@ -183,6 +191,37 @@ def embbag(tables, d: int, indices: np.ndarray, offsets: np.ndarray, batch: int,
     if skipped < 0:
         raise ValueError("oracle_embbag: bad arguments")
     return out, mag, int(skipped)
+
+
+KMEANS_ITERS = 10
+
+
+def quantize_rows_kmeans(x: np.ndarray, iters: int = KMEANS_ITERS, nthreads: int = 0, codes_ld: int | None = None):
+    """Codebook (per-row k-means) quantization: (codes uint8 [n, codes_ld], codebook
+    uint16 [n, 16] binary16 patterns, loss float32 [n])."""
+    x = np.asarray(x, dtype=np.float32)
+    if x.ndim != 2 or x.strides[1] != 4:
+        x = np.ascontiguousarray(x)
+    n, d = x.shape
+    ld = x.strides[0] // 4 if n > 1 else d
+    cld = (d + 1) // 2 if codes_ld is None else codes_ld
+    codes = np.zeros((n, cld), np.uint8)
+    cb = np.zeros((n, 16), np.uint16)
+    loss = np.zeros(n, np.float32)
+    rc = lib().oracle_quantize_rows_kmeans(_p(x), n, d, ld, _p(codes), cld, _p(cb), _p(loss), iters, nthreads)
+    if rc != 0:
+        raise ValueError("oracle_quantize_rows_kmeans: bad arguments")
+    return codes, cb, loss
+
+
+def dequantize_rows_kmeans(codes: np.ndarray, codebook: np.ndarray, d: int) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    cb = np.ascontiguousarray(codebook, dtype=np.uint16)
+    n = codes.shape[0]
+    out = np.zeros((n, d), np.float32)
+    if lib().oracle_dequantize_rows_kmeans(_p(codes), codes.shape[1], _p(cb), n, d, _p(out), d) != 0:
+        raise ValueError("oracle_dequantize_rows_kmeans: bad arguments")
+    return out
 
 
 BWD_WINDOW = 64

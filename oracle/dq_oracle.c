@@ -65,7 +65,21 @@
  *   e. Each touched row (one with at least one entry) is quantized again from its new
  *      master values by the quantizer above (greedy or min/max); other rows keep
  *      their codes.
- * *
+ * *   Codebook quantizer ("Post-Training 4-bit Quantization on Embedding Tables",
+ *   提出的方法 bullet 3: codebook quantization by k-means, values mapped to a
+ *   non-uniform set; 主要发现 bullet 3: the 18.8%-37.5% sizes fit 16 binary16 centroids
+ *   per row). The pages fix no initialisation, iteration count or precision; the
+ *   reading taken is one-dimensional Lloyd iterations in binary32:
+ *   K1. c_j = fma(j, fl(R / 15), xmin), j = 0..15 (the min/max quantizer's levels).
+ *   K2. `iters` times: a_k = the j minimising fl(|fl(x_k - c_j)|), ties to the lower j;
+ *       then for every j with n_j > 0 members, c_j = fl(S_j / n_j) with S_j the pairwise
+ *       sum (as the loss above) of x_k over the members (non-members add +0); an empty
+ *       cluster keeps its centroid.
+ *   K3. Stored centroids C_j = h(c_j); codes q_k = the j minimising fl(|fl(x_k - w(C_j))|),
+ *       ties to the lower j; packed as above. Row loss: the pairwise sum of
+ *       fl(fl(x_k - w(C_{q_k}))^2).
+ *   Dequantize: w(C_{q_k}); the codebook bag sums those values like the bag above.
+ *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fPIC -shared -pthread
  * (no FMA contraction and no excess precision, so every C operator below is one
  * IEEE binary32 operation; fmaf() is the C library's correctly rounded FMA).
@@ -320,6 +334,115 @@ float oracle_greedy_trace(const float *x, int32_t d, float *trace_lo, float *tra
 }
 
 /* ------------------------------------------------------------------------ */
+/* codebook quantizer (per-row k-means, 16 centroids)                       */
+/* ------------------------------------------------------------------------ */
+
+/* argmin_j fl(|fl(x - c_j)|), ties to the lower j */
+static int nearest(float x, const float *c)
+{
+    int best = 0;
+    float bd = fabsf(x - c[0]);
+    for (int j = 1; j < 16; j++) {
+        float dj = fabsf(x - c[j]);
+        if (dj < bd) {
+            bd = dj;
+            best = j;
+        }
+    }
+    return best;
+}
+
+/* Steps K1-K3 for one row; cbuf holds next_pow2(d) floats. Writes the stored
+ * centroids (binary16), the packed codes, and returns the row loss. */
+static float kmeans_row(const float *x, int d, int iters, float *cbuf, uint8_t *codes, uint16_t *codebook)
+{
+    float xmin = x[0], xmax = x[0];
+    for (int k = 1; k < d; k++) {
+        xmin = fminf(xmin, x[k]);
+        xmax = fmaxf(xmax, x[k]);
+    }
+    float step = (xmax - xmin) / ORACLE_LEVELS;
+    float c[16];
+    for (int j = 0; j < 16; j++)
+        c[j] = fmaf((float)j, step, xmin);
+    int P = next_pow2(d);
+    int a[ORACLE_MAX_D];
+    for (int it = 0; it < iters; it++) {
+        for (int k = 0; k < d; k++)
+            a[k] = nearest(x[k], c);
+        for (int j = 0; j < 16; j++) {
+            int n = 0;
+            for (int k = 0; k < P; k++) {
+                int member = k < d && a[k] == j;
+                cbuf[k] = member ? x[k] : 0.0f;
+                n += member;
+            }
+            if (n > 0)
+                c[j] = pairwise_sum(cbuf, P) / (float)n;
+        }
+    }
+    float C[16];
+    for (int j = 0; j < 16; j++) {
+        codebook[j] = oracle_f32_to_f16(c[j]);
+        C[j] = oracle_f16_to_f32(codebook[j]);
+    }
+    for (int m = 0; m < (d + 1) / 2; m++)
+        codes[m] = 0;
+    for (int k = 0; k < P; k++)
+        cbuf[k] = 0.0f;
+    for (int k = 0; k < d; k++) {
+        int q = nearest(x[k], C);
+        codes[k / 2] |= (uint8_t)(q << (4 * (k % 2)));
+        float e = x[k] - C[q];
+        cbuf[k] = e * e;
+    }
+    return pairwise_sum(cbuf, P);
+}
+
+typedef struct {
+    const float *x;
+    int64_t n, ld;
+    int d, iters;
+    uint8_t *codes;
+    int64_t codes_ld;
+    uint16_t *codebook;
+    float *loss;
+    int64_t begin, end;
+} kmeans_job;
+
+static void *kmeans_worker(void *arg)
+{
+    kmeans_job *j = (kmeans_job *)arg;
+    float cbuf[ORACLE_MAX_D];
+    for (int64_t r = j->begin; r < j->end; r++) {
+        float l = kmeans_row(j->x + r * j->ld, j->d, j->iters, cbuf, j->codes + r * j->codes_ld,
+                             j->codebook + 16 * r);
+        if (j->loss)
+            j->loss[r] = l;
+    }
+    return NULL;
+}
+
+/* K1-K3 for n rows (codebook [n][16] binary16 patterns); threaded over rows. */
+int32_t oracle_quantize_rows_kmeans(const float *x, int64_t n, int32_t d, int64_t ld, uint8_t *codes,
+                                    int64_t codes_ld, uint16_t *codebook, float *loss, int32_t iters,
+                                    int32_t nthreads);
+
+/* xhat_k = w(C_{q_k}) for n rows. */
+int32_t oracle_dequantize_rows_kmeans(const uint8_t *codes, int64_t codes_ld, const uint16_t *codebook, int64_t n,
+                                      int32_t d, float *out, int64_t out_ld)
+{
+    if (n < 0 || d < 1 || d > ORACLE_MAX_D || out_ld < d || codes_ld < (d + 1) / 2)
+        return -1;
+    for (int64_t r = 0; r < n; r++)
+        for (int k = 0; k < d; k++) {
+            int q = (codes[r * codes_ld + k / 2] >> (4 * (k % 2))) & 15;
+            out[r * out_ld + k] = oracle_f16_to_f32(codebook[16 * r + q]);
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
 /* threaded drivers                                                         */
 /* ------------------------------------------------------------------------ */
 
@@ -436,9 +559,10 @@ double oracle_row_l2_error(const float *x, int64_t n, int32_t d, int64_t x_ld, c
 
 typedef struct {
     const uint8_t *codes;
-    const uint16_t *scale_bias;
+    const uint16_t *scale_bias;     /* uniform rows: {scale, bias} per row */
     int64_t n_rows;
     int64_t codes_ld;
+    const uint16_t *codebook;       /* non-NULL: codebook rows, 16 binary16 centroids per row */
 } oracle_table;
 
 typedef struct {
@@ -470,12 +594,16 @@ static void *bag_worker(void *arg)
                 j->skipped++;
                 continue;
             }
-            float S = oracle_f16_to_f32(tab->scale_bias[2 * (int64_t)id]);
-            float Bv = oracle_f16_to_f32(tab->scale_bias[2 * (int64_t)id + 1]);
             const uint8_t *row = tab->codes + (int64_t)id * tab->codes_ld;
+            float S = 0.0f, Bv = 0.0f;
+            if (!tab->codebook) {
+                S = oracle_f16_to_f32(tab->scale_bias[2 * (int64_t)id]);
+                Bv = oracle_f16_to_f32(tab->scale_bias[2 * (int64_t)id + 1]);
+            }
             for (int k = 0; k < d; k++) {
                 int q = (row[k / 2] >> (4 * (k % 2))) & 0xf;
-                float xhat = fmaf((float)q, S, Bv);
+                float xhat = tab->codebook ? oracle_f16_to_f32(tab->codebook[16 * (int64_t)id + q])
+                                           : fmaf((float)q, S, Bv);
                 acc[k] += (double)xhat;
                 mag[k] += fabs((double)xhat);
             }
@@ -650,4 +778,29 @@ int64_t oracle_embbag(const oracle_table *tables, int32_t T, int32_t d, const in
     free(th);
     free(jobs);
     return skipped;
+}
+
+int32_t oracle_quantize_rows_kmeans(const float *x, int64_t n, int32_t d, int64_t ld, uint8_t *codes,
+                                    int64_t codes_ld, uint16_t *codebook, float *loss, int32_t iters,
+                                    int32_t nthreads)
+{
+    if (n < 0 || d < 1 || d > ORACLE_MAX_D || ld < d || codes_ld < (d + 1) / 2 || iters < 0)
+        return -1;
+    if (n == 0)
+        return 0;
+    int nt = resolve_threads(nthreads);
+    if (nt > n)
+        nt = (int)n;
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)nt);
+    kmeans_job *jobs = (kmeans_job *)malloc(sizeof(kmeans_job) * (size_t)nt);
+    for (int t = 0; t < nt; t++) {
+        kmeans_job j = {x, n, ld, d, iters, codes, codes_ld, codebook, loss, n * t / nt, n * (t + 1) / nt};
+        jobs[t] = j;
+        pthread_create(&th[t], NULL, kmeans_worker, &jobs[t]);
+    }
+    for (int t = 0; t < nt; t++)
+        pthread_join(th[t], NULL);
+    free(th);
+    free(jobs);
+    return 0;
 }
