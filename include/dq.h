@@ -166,6 +166,52 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
                           const uint8_t *codes, int64_t codes_ld, const uint16_t *scale_bias,
                           double *row_err, double *err_sum, void *cuda_stream);
 
+/*
+ * Codebook quantization (per-row k-means, 16 centroids): "Post-Training 4-bit
+ * Quantization on Embedding Tables", 提出的方法 (proposed method), bullet 3 (codebook
+ * quantization through k-means clustering, values mapped to a non-uniform set);
+ * 主要发现 (main findings), bullet 3 (its sizes, 18.8%-37.5% of FP32, fit 16 binary16
+ * centroids per row). Row format: the same d nibbles as above, and a codebook
+ * [n_rows][16] of binary16 bit patterns; element k decodes as codebook[q_k].
+ * The pages fix no algorithm details; this library computes, in binary32:
+ *   1. c_j = fma(j, (xmax - xmin) / 15, xmin), j = 0..15.
+ *   2. `iters` times: q_k = the j minimising |x_k - c_j| (ties to the lower j); for each
+ *      j with members, c_j = (pairwise sum of its members, padded with +0 as the loss
+ *      above) / (their count); a cluster without members keeps c_j.
+ *   3. codebook_j = fp16(c_j); codes = the nearest stored centroid (ties to the lower j);
+ *      row_loss = pairwise sum of (x_k - codebook[q_k])^2.
+ */
+#define DQ_KMEANS_MAX_ITERS 64
+
+/* dq_quantize_rows_kmeans4 -- arguments as dq_quantize_rows_int4, with codebook
+ * [n_rows][16] binary16 (output, 2-byte aligned), row_loss [n_rows] (nullable), iters in
+ * [0, DQ_KMEANS_MAX_ITERS]; d_flags: DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW. */
+dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld,
+                                   uint8_t *codes, int64_t codes_ld, uint16_t *codebook,
+                                   float *row_loss, int32_t iters, uint32_t *d_flags,
+                                   void *cuda_stream);
+
+/* dq_dequantize_rows_kmeans4 -- out[r][k] = codebook[r][q_k] (exact). */
+dq_status dq_dequantize_rows_kmeans4(const uint8_t *codes, int64_t codes_ld,
+                                     const uint16_t *codebook, int64_t n_rows, int32_t d,
+                                     float *out, int64_t out_ld, void *cuda_stream);
+
+/* One codebook-quantized table for the bag (device pointers). */
+typedef struct dq_kmeans_table {
+    const uint8_t *codes;
+    const uint16_t *codebook;  /* [n_rows][16] binary16 */
+    int64_t n_rows;
+    int64_t codes_ld;          /* >= (d+1)/2 */
+} dq_kmeans_table;
+
+/* dq_embbag_kmeans4_fwd -- the sum-pooled lookup of dq_embbag_int4_fwd over codebook
+ * tables: out[b][t*d + k] = binary32 sum, in id order, of codebook[id][q_k] over the
+ * bag (a bag of one id returns the dequantized row exactly). Same arguments, skips,
+ * clamping and flags as dq_embbag_int4_fwd. */
+dq_status dq_embbag_kmeans4_fwd(const dq_kmeans_table *tables, int32_t n_tables, int32_t d,
+                                const int32_t *indices, const int32_t *offsets, int32_t batch,
+                                float *out, uint32_t *d_flags, void *cuda_stream);
+
 /* One table of the bag backward: its binary32 master rows and their packed form.
  * All pointers are device pointers. */
 typedef struct dq_master_table {

@@ -10,9 +10,11 @@ raises DqError (build it with `python -m int4_row_wise_b200.build`).
 Low-level calls with the C names:
     dq_quantize_rows_int4, dq_dequantize_rows, dq_embbag_int4_fwd, dq_row_l2_error,
     dq_embbag_int4_bwd_workspace_bytes, dq_embbag_int4_bwd_sgd, dq_embbag_int4_bwd_sgd_noalloc,
+    dq_quantize_rows_kmeans4, dq_dequantize_rows_kmeans4, dq_embbag_kmeans4_fwd,
     dq_status_string, dq_last_error, dq_version
 Convenience wrappers that allocate their outputs with torch:
-    quantize_rows, dequantize_rows, embbag, row_l2_error, embbag_bwd_sgd
+    quantize_rows, dequantize_rows, embbag, row_l2_error, embbag_bwd_sgd,
+    quantize_rows_kmeans, dequantize_rows_kmeans, embbag_kmeans
 """
 from __future__ import annotations
 
@@ -29,6 +31,8 @@ __all__ = [
     "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_row_l2_error",
     "dq_embbag_int4_bwd_workspace_bytes", "dq_embbag_int4_bwd_sgd", "MasterTable",
     "dq_embbag_int4_bwd_sgd_noalloc", "DQ_BWD_STATIC_SCRATCH_BYTES",
+    "dq_quantize_rows_kmeans4", "dq_dequantize_rows_kmeans4", "dq_embbag_kmeans4_fwd", "KmeansTable",
+    "DQ_KMEANS_MAX_ITERS", "KMEANS_ITERS", "quantize_rows_kmeans", "dequantize_rows_kmeans", "embbag_kmeans",
     "dq_status_string", "dq_last_error", "dq_version",
     "quantize_rows", "dequantize_rows", "embbag", "row_l2_error", "embbag_bwd_sgd",
 ]
@@ -38,6 +42,8 @@ DQ_MODE_GREEDY, DQ_MODE_MINMAX = 0, 1
 DQ_FLAG_BAD_INDEX, DQ_FLAG_BAD_OFFSETS, DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW = 1, 2, 4, 8
 DQ_MAX_D, DQ_MAX_TABLES = 1024, 64
 DQ_BWD_STATIC_SCRATCH_BYTES = 32 << 20
+DQ_KMEANS_MAX_ITERS = 64
+KMEANS_ITERS = 10  # Lloyd iterations of the convenience wrapper
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libdq.so")
@@ -92,6 +98,12 @@ def load():
             L.dq_embbag_int4_bwd_sgd_noalloc.argtypes = [vp, i32, i32, vp, vp, i32, i64, vp, ctypes.c_float, i32,
                                                          vp, vp]
             L.dq_embbag_int4_bwd_sgd_noalloc.restype = ctypes.c_int
+            L.dq_quantize_rows_kmeans4.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, i32, vp, vp]
+            L.dq_quantize_rows_kmeans4.restype = ctypes.c_int
+            L.dq_dequantize_rows_kmeans4.argtypes = [vp, i64, vp, i64, i32, vp, i64, vp]
+            L.dq_dequantize_rows_kmeans4.restype = ctypes.c_int
+            L.dq_embbag_kmeans4_fwd.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp]
+            L.dq_embbag_kmeans4_fwd.restype = ctypes.c_int
             L.dq_status_string.argtypes, L.dq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
             L.dq_last_error.argtypes, L.dq_last_error.restype = [], ctypes.c_char_p
             L.dq_version.argtypes, L.dq_version.restype = [], i32
@@ -223,6 +235,48 @@ def dq_embbag_int4_bwd_sgd(tables: Sequence, d: int, indices, offsets, batch: in
     _check(st, "dq_embbag_int4_bwd_sgd")
 
 
+class _KmeansTable(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("codebook", ctypes.c_void_p),
+                ("n_rows", ctypes.c_int64), ("codes_ld", ctypes.c_int64)]
+
+
+class KmeansTable(NamedTuple):
+    """A codebook-quantized table on the device: codes uint8 [n, codes_ld], codebook int16
+    [n, 16] (binary16 bit patterns)."""
+    codes: object
+    codebook: object
+
+
+def dq_quantize_rows_kmeans4(x, n_rows: int, d: int, x_ld: int, codes, codes_ld: int, codebook, row_loss=None,
+                             iters: int = KMEANS_ITERS, d_flags=None, stream=None) -> None:
+    """C: dq_quantize_rows_kmeans4."""
+    st = load().dq_quantize_rows_kmeans4(_ptr(x), n_rows, d, x_ld, _ptr(codes), codes_ld, _ptr(codebook),
+                                         _ptr(row_loss), iters, _ptr(d_flags), _stream(stream))
+    _check(st, "dq_quantize_rows_kmeans4")
+
+
+def dq_dequantize_rows_kmeans4(codes, codes_ld: int, codebook, n_rows: int, d: int, out, out_ld: int,
+                               stream=None) -> None:
+    """C: dq_dequantize_rows_kmeans4."""
+    st = load().dq_dequantize_rows_kmeans4(_ptr(codes), codes_ld, _ptr(codebook), n_rows, d, _ptr(out), out_ld,
+                                           _stream(stream))
+    _check(st, "dq_dequantize_rows_kmeans4")
+
+
+def dq_embbag_kmeans4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, out, d_flags=None,
+                          stream=None) -> None:
+    """C: dq_embbag_kmeans4_fwd. tables: KmeansTable (or (codes, codebook)) per table."""
+    arr = (_KmeansTable * max(len(tables), 1))()
+    for t, tab in enumerate(tables):
+        codes, cb = tab[0], tab[1]
+        if codes.dim() != 2:
+            raise DqError(DQ_ERR_INVALID_ARG, "table codes must be a [n_rows, codes_ld] tensor")
+        arr[t] = _KmeansTable(_ptr(codes), _ptr(cb), int(codes.shape[0]), _row_stride(codes))
+    st = load().dq_embbag_kmeans4_fwd(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
+                                      _ptr(offsets), batch, _ptr(out), _ptr(d_flags), _stream(stream))
+    _check(st, "dq_embbag_kmeans4_fwd")
+
+
 def _master_array(tables):
     arr = (_MasterTable * max(len(tables), 1))()
     for t, tab in enumerate(tables):
@@ -312,3 +366,34 @@ def embbag_bwd_sgd(tables: Sequence, d: int, indices, offsets, batch: int, grad_
     dq_embbag_int4_bwd_sgd(tables, d, indices, offsets, batch, n, grad_out, lr, mode, workspace,
                            int(workspace.numel()), d_flags, stream)
     return workspace
+
+
+def quantize_rows_kmeans(x, iters: int = KMEANS_ITERS, with_loss: bool = True, d_flags=None, stream=None):
+    """Codebook quantization of x (CUDA float32 [n, d], unit stride along d). Returns
+    (codes uint8 [n, codes_ld], codebook int16 [n, 16], row_loss float32 [n] or None)."""
+    import torch
+    if x.dim() != 2 or x.dtype != torch.float32 or (x.shape[0] > 1 and x.stride(1) != 1):
+        raise DqError(DQ_ERR_INVALID_ARG, "x must be a float32 [n, d] tensor with unit stride along d")
+    n, d = x.shape
+    cld = _codes_ld(d)
+    codes = torch.empty((n, cld), dtype=torch.uint8, device=x.device)
+    cb = torch.empty((n, 16), dtype=torch.int16, device=x.device)
+    loss = torch.empty(n, dtype=torch.float32, device=x.device) if with_loss else None
+    dq_quantize_rows_kmeans4(x, n, d, x.stride(0) if n > 1 else d, codes, cld, cb, loss, iters, d_flags, stream)
+    return codes, cb, loss
+
+
+def dequantize_rows_kmeans(codes, codebook, d: int, stream=None):
+    import torch
+    n = codes.shape[0]
+    out = torch.empty((n, d), dtype=torch.float32, device=codes.device)
+    dq_dequantize_rows_kmeans4(codes, _row_stride(codes) if n else codes.shape[1], codebook, n, d, out, d, stream)
+    return out
+
+
+def embbag_kmeans(tables: Sequence, d: int, indices, offsets, batch: int, d_flags=None, stream=None):
+    """Sum-pooled lookup over codebook tables; returns float32 [batch, len(tables) * d]."""
+    import torch
+    out = torch.empty((batch, len(tables) * d), dtype=torch.float32, device=indices.device)
+    dq_embbag_kmeans4_fwd(tables, d, indices, offsets, batch, out, d_flags, stream)
+    return out

@@ -211,6 +211,105 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
     return launched(dq::launch_row_l2(a, sms, (cudaStream_t)cuda_stream), "row_l2_error");
 }
 
+dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, uint8_t *codes,
+                                   int64_t codes_ld, uint16_t *codebook, float *row_loss, int32_t iters,
+                                   uint32_t *d_flags, void *cuda_stream)
+{
+    if (n_rows < 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (x_ld < d)
+        return fail(DQ_ERR_INVALID_ARG, "x_ld = %lld < d = %d", (long long)x_ld, d);
+    if (codes_ld < (d + 1) / 2)
+        return fail(DQ_ERR_INVALID_ARG, "codes_ld = %lld < (d+1)/2 = %d", (long long)codes_ld, (d + 1) / 2);
+    if (iters < 0 || iters > DQ_KMEANS_MAX_ITERS)
+        return fail(DQ_ERR_INVALID_ARG, "iters = %d outside [0, %d]", iters, DQ_KMEANS_MAX_ITERS);
+    if (n_rows > 0 && (!x || !codes || !codebook))
+        return fail(DQ_ERR_INVALID_ARG, "x, codes and codebook must be non-NULL when n_rows > 0");
+    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(codebook) & 1)))
+        return fail(DQ_ERR_INVALID_ARG, "x must be 4-byte and codebook 2-byte aligned");
+    if (n_rows == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::KmeansArgs a{x, n_rows, x_ld, d, iters, codes, codes_ld, codebook, row_loss, d_flags};
+    return launched(dq::launch_kmeans(a, (cudaStream_t)cuda_stream), "quantize_rows_kmeans4");
+}
+
+dq_status dq_dequantize_rows_kmeans4(const uint8_t *codes, int64_t codes_ld, const uint16_t *codebook,
+                                     int64_t n_rows, int32_t d, float *out, int64_t out_ld, void *cuda_stream)
+{
+    if (n_rows < 0)
+        return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (codes_ld < (d + 1) / 2)
+        return fail(DQ_ERR_INVALID_ARG, "codes_ld = %lld < (d+1)/2 = %d", (long long)codes_ld, (d + 1) / 2);
+    if (out_ld < d)
+        return fail(DQ_ERR_INVALID_ARG, "out_ld = %lld < d = %d", (long long)out_ld, d);
+    if (n_rows > 0 && (!codes || !codebook || !out))
+        return fail(DQ_ERR_INVALID_ARG, "codes, codebook and out must be non-NULL when n_rows > 0");
+    if (n_rows == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::KmeansDequantArgs a{codes, codes_ld, codebook, n_rows, d, out, out_ld};
+    return launched(dq::launch_kmeans_dequantize(a, sms, (cudaStream_t)cuda_stream), "dequantize_rows_kmeans4");
+}
+
+dq_status dq_embbag_kmeans4_fwd(const dq_kmeans_table *tables, int32_t n_tables, int32_t d, const int32_t *indices,
+                                const int32_t *offsets, int32_t batch, float *out, uint32_t *d_flags,
+                                void *cuda_stream)
+{
+    if (n_tables < 1 || n_tables > DQ_MAX_TABLES)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables = %d outside [1, %d]", n_tables, DQ_MAX_TABLES);
+    if (!tables)
+        return fail(DQ_ERR_INVALID_ARG, "tables must be non-NULL");
+    if (d < 1 || d > DQ_MAX_D)
+        return fail(DQ_ERR_INVALID_ARG, "d = %d outside [1, %d]", d, DQ_MAX_D);
+    if (batch < 0)
+        return fail(DQ_ERR_INVALID_ARG, "batch = %d < 0", batch);
+    if ((int64_t)n_tables * batch + 1 > INT32_MAX)
+        return fail(DQ_ERR_INVALID_ARG, "n_tables * batch + 1 offsets exceed int32 indexing");
+    dq::KmeansBagTables tabs;
+    memset(&tabs, 0, sizeof tabs);
+    for (int t = 0; t < n_tables; ++t) {
+        const dq_kmeans_table &tb = tables[t];
+        if (tb.n_rows < 0)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].n_rows = %lld < 0", t, (long long)tb.n_rows);
+        if (tb.codes_ld < (d + 1) / 2)
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d].codes_ld = %lld < (d+1)/2 = %d", t,
+                        (long long)tb.codes_ld, (d + 1) / 2);
+        if (tb.n_rows > 0 && (!tb.codes || !tb.codebook))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codes and codebook must be non-NULL", t);
+        tabs.codes[t] = tb.codes;
+        tabs.codebook[t] = tb.codebook;
+        tabs.n_rows[t] = tb.n_rows;
+        tabs.codes_ld[t] = tb.codes_ld;
+    }
+    if (batch > 0 && (!indices || !offsets || !out))
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
+    if (batch == 0)
+        return ok();
+    int sms = 0;
+    dq_status st = current_device(&sms);
+    if (st != DQ_OK)
+        return st;
+    if (fault_injected())
+        return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
+    dq::KmeansBagArgs a{n_tables, d, batch, indices, offsets, out, d_flags, dq::make_batch_div((uint32_t)batch)};
+    return launched(dq::launch_kmeans_bag(tabs, a, sms, (cudaStream_t)cuda_stream), "embbag_kmeans4");
+}
+
 size_t dq_embbag_int4_bwd_workspace_bytes(int32_t d, int64_t n_indices)
 {
     if (d < 1 || d > DQ_MAX_D || n_indices < 0 || n_indices > INT32_MAX)

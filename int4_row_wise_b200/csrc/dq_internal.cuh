@@ -116,6 +116,44 @@ struct BwdArgs {
     uint32_t *flags;
 };
 
+// Codebook (per-row k-means) quantizer, dequantization and bag.
+struct KmeansArgs {
+    const float *x;
+    int64_t n, ld;
+    int d, iters;
+    uint8_t *codes;
+    int64_t codes_ld;
+    uint16_t *codebook;        // [n][16] binary16
+    float *row_loss;
+    uint32_t *flags;
+};
+
+struct KmeansDequantArgs {
+    const uint8_t *codes;
+    int64_t codes_ld;
+    const uint16_t *codebook;
+    int64_t n;
+    int d;
+    float *out;
+    int64_t out_ld;
+};
+
+struct KmeansBagTables {
+    const uint8_t *codes[DQ_MAX_TABLES];
+    const uint16_t *codebook[DQ_MAX_TABLES];
+    int64_t n_rows[DQ_MAX_TABLES];
+    int64_t codes_ld[DQ_MAX_TABLES];
+};
+
+struct KmeansBagArgs {
+    int T, d, batch;
+    const int32_t *indices;
+    const int32_t *offsets;
+    float *out;
+    uint32_t *flags;
+    BatchDiv div;
+};
+
 // Byte offsets of the pieces of the backward's workspace (each 256-byte aligned).
 struct BwdLayout {
     size_t hdr, keys0, keys1, bags0, bags1, hist, totals, partials, span_slot, list, grad_rows, total;
@@ -146,6 +184,9 @@ cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t st
 cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_kmeans(const KmeansArgs &a, cudaStream_t stream);
+cudaError_t launch_kmeans_dequantize(const KmeansDequantArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_requant(const RequantArgs &a, int64_t max_rows, int mode, int num_sms, cudaStream_t stream);
 
 // Sets the calling thread's dq_last_error() text (for entry points outside dq_api.cu).

@@ -1,0 +1,305 @@
+// dq_kmeans.cu -- codebook 4-bit quantization (per-row k-means, 16 centroids), its
+// dequantization and its sum-pooled bag, on sm_100a.
+//
+// "Post-Training 4-bit Quantization on Embedding Tables" (Guan et al., 2019), review
+// page, section 提出的方法 (proposed method), bullet 3: codebook quantization through
+// k-means clustering maps a row's values to a non-uniform set; section 主要发现 (main
+// findings), bullet 3: it gives the lowest normalized l2 loss at 18.8%-37.5% of the
+// FP32 size (16 binary16 centroids and d nibbles per row). The steps (dq.h states them):
+// centroids start at the 16 levels of the min/max quantizer, `iters` Lloyd iterations
+// in binary32 (nearest centroid by |x - c|, ties to the lower index; the mean of a
+// cluster = its pairwise member sum / its size; an empty cluster keeps its centroid),
+// binary16 storage, final codes against the stored centroids.
+//
+// Layout as the greedy quantizer's: a row of d <= P = next_pow2(d) elements in
+// registers, W lanes per row, M = P / W contiguous elements per lane. A cluster's
+// member sum is the pairwise (recursive-halving) sum over the padded row: each lane
+// builds the tree of its aligned block bottom-up, and an XOR butterfly over the W
+// lanes joins the blocks in tree order; IEEE addition is commutative, so every lane
+// of a row ends with the identical sums and centroids. ALU bound: each iteration
+// costs 16 distance evaluations and 16 masked adds per element.
+#include <cfloat>
+
+#include "dq_internal.cuh"
+
+namespace dq {
+namespace {
+
+constexpr float kLevels = 15.0f;
+
+// Pairwise sum of v[0..M) (M a power of two), bottom-up: the recursive-halving tree.
+template <int M>
+__device__ __forceinline__ float block_pairwise(float (&v)[M])
+{
+#pragma unroll
+    for (int s = 1; s < M; s <<= 1) {
+#pragma unroll
+        for (int i = 0; i < M; i += 2 * s)
+            v[i] = __fadd_rn(v[i], v[i + s]);
+    }
+    return v[0];
+}
+
+template <int W>
+__device__ __forceinline__ float row_pairwise(float lane_sum)
+{
+#pragma unroll
+    for (int o = 1; o < W; o <<= 1)
+        lane_sum = __fadd_rn(lane_sum, __shfl_xor_sync(0xffffffffu, lane_sum, o));
+    return lane_sum;
+}
+
+template <int W>
+__device__ __forceinline__ int row_count(int c)
+{
+#pragma unroll
+    for (int o = 1; o < W; o <<= 1)
+        c += __shfl_xor_sync(0xffffffffu, c, o);
+    return c;
+}
+
+// argmin_j fl(|fl(x - c_j)|), ties to the lower j
+__device__ __forceinline__ int nearest16(float x, const float (&c)[16])
+{
+    int best = 0;
+    float bd = fabsf(__fsub_rn(x, c[0]));
+#pragma unroll
+    for (int j = 1; j < 16; ++j) {
+        const float dj = fabsf(__fsub_rn(x, c[j]));
+        const bool better = dj < bd;
+        bd = better ? dj : bd;
+        best = better ? j : best;
+    }
+    return best;
+}
+
+// One row per W lanes, M contiguous elements per lane; FULL: d == M * W.
+template <int M, int W, bool FULL>
+__global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
+{
+    const int sub = threadIdx.x & (W - 1);
+    int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / W;
+    const bool active = row < a.n;
+    if (!active)
+        row = a.n - 1;  // idle lanes shadow the last row so the warp stays converged
+    const int d = a.d;
+    const int kbase = sub * M;
+    const float *xr = a.x + row * a.ld + kbase;
+    float x[M];
+    bool nonfinite = false;
+    float mn = FLT_MAX, mx = -FLT_MAX;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const bool ok = FULL || kbase + m < d;
+        x[m] = ok ? __ldg(xr + m) : 0.0f;
+        if (ok) {
+            mn = fminf(mn, x[m]);
+            mx = fmaxf(mx, x[m]);
+            nonfinite |= !isfinite(x[m]);
+        }
+    }
+#pragma unroll
+    for (int o = 1; o < W; o <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    // K1: the min/max levels
+    const float step = __fdiv_rn(__fsub_rn(mx, mn), kLevels);
+    float c[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        c[j] = __fmaf_rn((float)j, step, mn);
+    // K2: Lloyd iterations
+    uint8_t q[M];
+    for (int it = 0; it < a.iters; ++it) {
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            q[m] = (uint8_t)nearest16(x[m], c);
+        float s[16];
+        int n[16];
+#pragma unroll 16
+        for (int j = 0; j < 16; ++j) {
+            float v[M];
+            int cnt = 0;
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                const bool member = (FULL || kbase + m < d) && q[m] == j;
+                v[m] = member ? x[m] : 0.0f;
+                cnt += member;
+            }
+            s[j] = row_pairwise<W>(block_pairwise<M>(v));
+            n[j] = row_count<W>(cnt);
+        }
+#pragma unroll 16
+        for (int j = 0; j < 16; ++j)
+            c[j] = n[j] > 0 ? __fdiv_rn(s[j], (float)n[j]) : c[j];
+    }
+    // K3: binary16 centroids, final codes, loss
+    float C[16];
+    __half h[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        h[j] = __float2half_rn(c[j]);
+        C[j] = __half2float(h[j]);
+    }
+    float e2[M];
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const bool ok = FULL || kbase + m < d;
+        q[m] = ok ? (uint8_t)nearest16(x[m], C) : (uint8_t)0;
+        float cq = C[0];
+#pragma unroll
+        for (int j = 1; j < 16; ++j)
+            cq = q[m] == j ? C[j] : cq;
+        const float e = __fsub_rn(x[m], cq);
+        e2[m] = ok ? __fmul_rn(e, e) : 0.0f;
+    }
+    const float loss = row_pairwise<W>(block_pairwise<M>(e2));
+    if (!active)
+        return;
+    uint8_t *cr = a.codes + row * a.codes_ld + kbase / 2;
+#pragma unroll
+    for (int m = 0; m < (M + 1) / 2; ++m) {
+        const int k0 = 2 * m;
+        if (FULL || kbase + k0 < d) {
+            const unsigned lo = q[k0];
+            const unsigned hi = (k0 + 1 < M) ? q[k0 + 1] : 0u;
+            cr[m] = (uint8_t)(lo | (hi << 4));
+        }
+    }
+    if (sub == 0) {
+        uint16_t *cb = a.codebook + 16 * row;
+        bool over = false;
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            cb[j] = __half_as_ushort(h[j]);
+            over |= isinf(C[j]);
+        }
+        if (a.row_loss)
+            a.row_loss[row] = loss;
+        if (over)
+            raise_flag(a.flags, DQ_FLAG_FP16_OVERFLOW);
+    }
+    if (nonfinite)
+        raise_flag(a.flags, DQ_FLAG_NONFINITE);
+}
+
+template <int M, int W>
+cudaError_t launch_kmeans_mw(const KmeansArgs &a, cudaStream_t stream)
+{
+    constexpr int kBlock = 128;
+    const int64_t grid = (a.n * W + kBlock - 1) / kBlock;
+    if (a.d == M * W)
+        kmeans_rows_kernel<M, W, true><<<(unsigned)grid, kBlock, 0, stream>>>(a);
+    else
+        kmeans_rows_kernel<M, W, false><<<(unsigned)grid, kBlock, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+// xhat = w(C[q]): one thread per pair of elements.
+__global__ void __launch_bounds__(256) kmeans_dequant_kernel(const KmeansDequantArgs a)
+{
+    const int pairs = (a.d + 1) / 2;
+    const int64_t total = a.n * pairs;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / pairs;
+        const int m = (int)(i - r * pairs);
+        const unsigned byte = __ldg(a.codes + r * a.codes_ld + m);
+        const uint16_t *cb = a.codebook + 16 * r;
+        float *o = a.out + r * a.out_ld + 2 * m;
+        o[0] = __half2float(__ushort_as_half(__ldg(cb + (byte & 15u))));
+        if (2 * m + 1 < a.d)
+            o[1] = __half2float(__ushort_as_half(__ldg(cb + (byte >> 4))));
+    }
+}
+
+// One warp per bag (t, b); lane l owns elements l, l + 32, ...; per id, lanes 0..15 read
+// the row's 16 centroids and each lane takes its element's centroid by shuffle. The
+// sum runs in binary32 in id order, so a bag of one id returns the dequantized row.
+__global__ void __launch_bounds__(256) kmeans_bag_kernel(const KmeansBagTables tabs, const KmeansBagArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t G = (int64_t)a.T * a.batch;
+    const int32_t total = a.offsets[G];
+    const int chunks = (a.d + 31) / 32;
+    for (int64_t g = warp; g < G; g += warps) {
+        const int t = (int)div_batch((uint32_t)g, a.div);
+        const int64_t b = g - (int64_t)t * a.batch;
+        int32_t p0 = a.offsets[g], p1 = a.offsets[g + 1];
+        p0 = p0 < 0 ? 0 : (p0 > total ? total : p0);
+        p1 = p1 < 0 ? 0 : (p1 > total ? total : p1);
+        if (p1 < p0) {
+            if (lane == 0)
+                raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
+            p1 = p0;
+        }
+        const int64_t n_rows = tabs.n_rows[t];
+        float *out = a.out + b * (int64_t)a.T * a.d + (int64_t)t * a.d;
+        for (int ch = 0; ch < chunks; ++ch) {
+            const int k = ch * 32 + lane;
+            float acc = 0.0f;
+            for (int32_t p = p0; p < p1; ++p) {
+                const int32_t id = __ldg(a.indices + p);
+                if (id < 0 || id >= n_rows) {
+                    if (lane == 0 && ch == 0)
+                        raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                    continue;
+                }
+                const float cj = lane < 16 ? __half2float(__ushort_as_half(__ldg(tabs.codebook[t] + 16 * (int64_t)id + lane)))
+                                           : 0.0f;
+                unsigned qk = 0;
+                if (k < a.d)
+                    qk = (__ldg(tabs.codes[t] + (int64_t)id * tabs.codes_ld[t] + k / 2) >> (4 * (k & 1))) & 15u;
+                const float v = __shfl_sync(0xffffffffu, cj, (int)qk);
+                acc = __fadd_rn(acc, v);
+            }
+            if (k < a.d)
+                out[k] = acc;
+        }
+    }
+}
+
+} // namespace
+
+cudaError_t launch_kmeans(const KmeansArgs &a, cudaStream_t stream)
+{
+    int p = 1;
+    while (p < a.d)
+        p <<= 1;
+    switch (p) {
+    case 1: return launch_kmeans_mw<1, 1>(a, stream);
+    case 2: return launch_kmeans_mw<2, 1>(a, stream);
+    case 4: return launch_kmeans_mw<4, 1>(a, stream);
+    case 8: return launch_kmeans_mw<8, 1>(a, stream);
+    case 16: return launch_kmeans_mw<16, 1>(a, stream);
+    case 32: return launch_kmeans_mw<16, 2>(a, stream);
+    case 64: return launch_kmeans_mw<16, 4>(a, stream);
+    case 128: return launch_kmeans_mw<16, 8>(a, stream);
+    case 256: return launch_kmeans_mw<16, 16>(a, stream);
+    case 512: return launch_kmeans_mw<16, 32>(a, stream);
+    case 1024: return launch_kmeans_mw<32, 32>(a, stream);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_kmeans_dequantize(const KmeansDequantArgs &a, int num_sms, cudaStream_t stream)
+{
+    const int64_t total = a.n * ((a.d + 1) / 2);
+    const int64_t need = (total + 255) / 256;
+    const int64_t cap = (int64_t)num_sms * 16;
+    kmeans_dequant_kernel<<<(unsigned)(need < cap ? need : cap), 256, 0, stream>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &a, int num_sms, cudaStream_t stream)
+{
+    const int64_t G = (int64_t)a.T * a.batch;
+    const int64_t need = (G * 32 + 255) / 256;
+    const int64_t cap = (int64_t)num_sms * 16;
+    kmeans_bag_kernel<<<(unsigned)(need < cap ? need : cap), 256, 0, stream>>>(tabs, a);
+    return cudaGetLastError();
+}
+
+} // namespace dq

@@ -158,3 +158,30 @@ def test_embbag_bwd_no_entries_is_a_noop_and_workspace_size(L):
     assert small % 256 == 0 and big % 256 == 0
     # keys, bags (twice each), list: 20 B; G rows: 4 d B; window parts: d / 4 B per entry
     assert 10 ** 6 * (20 + 4 * 64 + 64 // 4) <= big <= 10 ** 6 * (20 + 4 * 64 + 64 // 4) + 10 ** 6
+
+
+@pytest.mark.parametrize("args,msg", [
+    ((NULL, -1, 16, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "n_rows"),
+    ((NULL, 4, 0, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "d = 0"),
+    ((NULL, 4, 16, 15, NULL, 8, NULL, NULL, 10, NULL, NULL), "x_ld"),
+    ((NULL, 4, 16, 16, NULL, 7, NULL, NULL, 10, NULL, NULL), "codes_ld"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, 65, NULL, NULL), "iters"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, -1, NULL, NULL), "iters"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "non-NULL"),
+])
+def test_kmeans_quantize_rejects(L, args, msg):
+    assert L.dq_quantize_rows_kmeans4(*args) == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
+def test_kmeans_dequantize_and_bag_reject(L):
+    assert L.dq_dequantize_rows_kmeans4(None, 8, None, 3, 16, None, 15, None) == dq.DQ_ERR_INVALID_ARG
+    assert "out_ld" in L.dq_last_error().decode()
+    arr = (dq._KmeansTable * 1)(dq._KmeansTable(None, None, 10, 8))
+    p = ctypes.cast(arr, ctypes.c_void_p)
+    assert L.dq_embbag_kmeans4_fwd(p, 1, 16, None, None, 4, None, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "codebook" in L.dq_last_error().decode()
+    assert L.dq_embbag_kmeans4_fwd(p, 1, 16, None, None, 0, None, None, None) == dq.DQ_ERR_INVALID_ARG
+    arr0 = (dq._KmeansTable * 1)(dq._KmeansTable(None, None, 0, 8))
+    assert L.dq_embbag_kmeans4_fwd(ctypes.cast(arr0, ctypes.c_void_p), 1, 16, None, None, 0, None, None,
+                                   None) == dq.DQ_OK
