@@ -555,6 +555,105 @@ def run_bwd(args, wl: W.Workload) -> None:
         "clocks": clk, "gpu_launches": launches * args.steps}), flush=True)
 
 
+def run_codebook(args, wl: W.Workload) -> None:
+    """Times the codebook quantizer (per-row k-means, 16 binary16 centroids): one step =
+    quantize every table of the workload + one codebook lookup call, inputs resident in
+    HBM. Reports rows/s, the quantizer's ALU roofline, the lookup's unique bytes/s, and
+    the normalized l2 error of the codebook and the greedy uniform quantizer on the first
+    rows of the largest table."""
+    import torch
+    import int4_row_wise_b200 as dq
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    dq.load()
+    big = wl.total_rows * wl.d * 4 > LARGE_BYTES
+    xs = []
+    for t in range(wl.n_tables):
+        if big:
+            st = W.SharedTable(wl, t)
+            xs.append(torch.from_numpy(st.array).to(dev))
+            st.close()
+        else:
+            xs.append(torch.from_numpy(W.table_rows(wl, t)).to(dev))
+    d = wl.d
+    cld = dq._codes_ld(d)
+    iters = dq.KMEANS_ITERS
+    codes = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wl.rows]
+    cbs = [torch.empty((n, 16), dtype=torch.int16, device=dev) for n in wl.rows]
+    tables = [dq.KmeansTable(c, b) for c, b in zip(codes, cbs)]
+    n_batches = 4
+    bh = [W.lookup_batch(wl, batch_id=i) for i in range(n_batches)]
+    bd = [(torch.from_numpy(i).to(dev), torch.from_numpy(o).to(dev)) for i, o in bh]
+    rb = (d + 1) // 2 + 32
+    nbytes = []
+    for i, o in bh:
+        uniq = sum(np.unique(i[o[t * wl.batch]:o[(t + 1) * wl.batch]]).size for t in range(wl.n_tables))
+        nbytes.append(uniq * rb + i.nbytes + o.nbytes + wl.batch * wl.n_tables * d * 4)
+    out = torch.empty((wl.batch, wl.n_tables * d), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(k, ev=None):
+        if ev:
+            ev[0].record(stream)
+        for t, x in enumerate(xs):
+            if wl.rows[t]:
+                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, codes[t], cld, cbs[t], None, iters, None, stream)
+        if ev:
+            ev[1].record(stream)
+        i, o = bd[k % n_batches]
+        dq.dq_embbag_kmeans4_fwd(tables, d, i, o, wl.batch, out, None, stream)
+        if ev:
+            ev[2].record(stream)
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize(dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with ClockSampler(0) as clocks:
+        for k in range(args.steps):
+            step(k, evs[k])
+        torch.cuda.synchronize(dev)
+    clk = clocks.summary()
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    b_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    tot_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
+    rows = wl.total_rows * args.steps
+    # algorithmic work per element: per iteration 16 distances (subtract, compare) and one
+    # add into the element's own cluster; then the final 16 distances and the loss terms
+    flops = wl.total_rows * d * (iters * 33 + 35) * args.steps
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    peak = FP32_LANES_PER_SM * sms * 1965e6 / 1e12  # one FP32 op per lane per clock (no FMA here)
+    achieved = flops / (q_ms / 1e3) / 1e12
+    bag_gbs = sum(nbytes[k % n_batches] for k in range(args.steps)) / (b_ms / 1e3) / 1e9
+    # quality on the first rows of the largest table
+    t = int(np.argmax(wl.rows))
+    n_q = min(wl.rows[t], 200000)
+    x = xs[t][:n_q]
+    xk = dq.dequantize_rows_kmeans(codes[t][:n_q], cbs[t][:n_q], d)
+    uc, usb, _, _ = dq.quantize_rows(x, with_loss=False)
+    xu = dq.dequantize_rows(uc, usb, d)
+    x64 = x.double()
+    nrm = x64.norm(dim=1)
+    ok = nrm > 0
+    l2k = float(((x64 - xk.double()).norm(dim=1)[ok] / nrm[ok]).mean())
+    l2u = float(((x64 - xu.double()).norm(dim=1)[ok] / nrm[ok]).mean())
+    print(json.dumps({
+        "metric": "codebook (k-means, 16 binary16 centroids) 4-bit quantization rows/s, step = quantize all tables "
+                  "+ one codebook lookup call",
+        "value": rows / (tot_ms / 1e3), "unit": "rows/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_ms / args.steps, "higher_is_better": True, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": _workload_desc(wl), "lloyd_iterations": iters,
+                   "l2": "inputs larger than L2 (fp32 tables %.0f MB > 126 MB)" % (wl.total_rows * d * 4 / 1e6)},
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{FP32_LANES_PER_SM} FP32 lanes x {sms} SMs x 1965 MHz, one op per lane-clock",
+                     "flops_per_element": iters * 33 + 35},
+        "embbag": {"achieved": bag_gbs, "unit": "GB/s", "peak": _measured_hbm(), "frac": bag_gbs / _measured_hbm(),
+                   "ms_per_call": b_ms / args.steps},
+        "quality": {"normalized_l2_codebook": l2k, "normalized_l2_greedy_uniform": l2u, "rows": n_q,
+                    "bytes_per_row_codebook": rb, "bytes_per_row_uniform": (d + 1) // 2 + 4},
+        "clocks": clk, "gpu_launches": (sum(1 for n in wl.rows if n) + 1) * args.steps}), flush=True)
+
+
 def _measured_hbm() -> float:
     try:
         return float(json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"])
@@ -654,6 +753,8 @@ def main(argv=None) -> None:
     ap.add_argument("--lookup-only", action="store_true",
                     help="time only the lookup, over random packed tables of the workload's sizes")
     ap.add_argument("--streams", type=int, default=4, help="streams the per-table quantize launches spread over")
+    ap.add_argument("--codebook", action="store_true",
+                    help="time the codebook (k-means) quantizer and its lookup on the workload's tables")
     ap.add_argument("--bwd", action="store_true",
                     help="time the bag backward + SGD + re-quantization over masters of the workload's sizes")
     args = ap.parse_args(argv)
@@ -666,6 +767,8 @@ def main(argv=None) -> None:
         run_lookup_only(args, wl)
     elif args.bwd:
         run_bwd(args, wl)
+    elif args.codebook:
+        run_codebook(args, wl)
     else:
         run_gpu(args, wl)
 
