@@ -388,6 +388,11 @@ def run_gpu(args, wl: W.Workload) -> None:
     bag_gbs = sum(bag_bytes[k % n_batches] for k in range(args.steps)) / (bag_ms / 1e3) / 1e9
     hbm = _measured_hbm()
 
+    # --- the widened rows, after the timed region, on the same device tables
+    next_rows = None
+    if rank == 0 and not args.no_next_rows:
+        next_rows = _next_rows(wlr, xs, codes, sbs, batches_h, batches, dev, stream, dq)
+
     # --- end to end through the public API with pinned host buffers
     e2e = None
     if rank == 0 and not args.no_e2e:
@@ -416,6 +421,7 @@ def run_gpu(args, wl: W.Workload) -> None:
                        "peak_source": "MEASURED_PEAKS.json hbm_gbs (of measured)"},
             "quality": quality,
             "l2_eval": l2_eval,
+            "next_rows": next_rows,
             "phases_ms_per_step": {"quantize": q_ms / args.steps, "embbag": bag_ms / args.steps,
                                    "dequantize": dq_ms / args.steps},
             "gpu_launches": launches_per_step * args.steps,
@@ -427,6 +433,94 @@ def run_gpu(args, wl: W.Workload) -> None:
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def _next_rows(wl, xs, codes, sbs, batches_h, batches, dev, stream, dq) -> dict:
+    """The codebook quantizer (all tables, 3 steps, then one codebook lookup per step) and
+    the bag backward + SGD + re-quantization (10 calls over the step's lookup batches,
+    each with its own seeded output gradient), timed with CUDA events after the bench's
+    timed region. The codebook leg runs first, on the untouched tables; the backward then
+    updates the tables in place (nothing after it reads them)."""
+    import torch
+    d = wl.d
+    cld = dq._codes_ld(d)
+    T, B = wl.n_tables, wl.batch
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    out = {}
+    # codebook quantizer + its lookup
+    kc = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wl.rows]
+    kcb = [torch.empty((n, 16), dtype=torch.int16, device=dev) for n in wl.rows]
+    kt = [dq.KmeansTable(c, b) for c, b in zip(kc, kcb)]
+    bag_out = torch.empty((B, T * d), dtype=torch.float32, device=dev)
+    iters = dq.KMEANS_ITERS
+
+    def cb_step(k):
+        for t, x in enumerate(xs):
+            if wl.rows[t]:
+                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, kc[t], cld, kcb[t], None, iters, None, stream)
+        i, o = batches[k % len(batches)]
+        dq.dq_embbag_kmeans4_fwd(kt, d, i, o, B, bag_out, None, stream)
+
+    cb_step(0)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for k in range(3):
+        cb_step(k)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    cb_ms = e0.elapsed_time(e1) / 3
+    t = int(np.argmax(wl.rows))
+    n_q = min(wl.rows[t], 200000)
+    x = xs[t][:n_q]
+    xk = dq.dequantize_rows_kmeans(kc[t][:n_q], kcb[t][:n_q], d).double()
+    xu = dq.dequantize_rows(codes[t][:n_q], sbs[t][:n_q], d).double()
+    x64 = x.double()
+    nrm = x64.norm(dim=1)
+    ok = nrm > 0
+    cb_flops = wl.total_rows * d * (iters * 33 + 35)
+    cb_peak = FP32_LANES_PER_SM * sms * 1965e6 / 1e12
+    out["codebook"] = {
+        "what": "codebook 4-bit quantization (per-row k-means, 16 binary16 centroids, "
+                f"{iters} Lloyd iterations) of all tables + one codebook lookup call",
+        "rows_per_s": wl.total_rows / (cb_ms / 1e3), "ms_per_step": cb_ms,
+        "alu_frac_upper": cb_flops / (cb_ms / 1e3) / 1e12 / cb_peak,
+        "alu_peak_tops": cb_peak,
+        "normalized_l2_codebook": float(((x64 - xk).norm(dim=1)[ok] / nrm[ok]).mean()),
+        "normalized_l2_greedy": float(((x64 - xu).norm(dim=1)[ok] / nrm[ok]).mean()),
+        "bytes_per_row": {"codebook": (d + 1) // 2 + 32, "greedy": (d + 1) // 2 + 4}}
+    del kc, kcb, kt, xk, xu, x64
+    # bag backward + SGD on the tables as binary32 masters + re-quantization of touched rows
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4321)
+    grads = [torch.randn((B, T * d), generator=gen, device=dev) * 1e-2 for _ in batches]
+    n_ids = [int(i.size) for i, _ in batches_h]
+    touched = [_touched_rows(wl, i, o) for i, o in batches_h]
+    ws = torch.empty(max(dq.dq_embbag_int4_bwd_workspace_bytes(d, max(n_ids)), 256), dtype=torch.uint8,
+                     device=dev)
+    mt = [dq.MasterTable(x_, c_, s_) for x_, c_, s_ in zip(xs, codes, sbs)]
+
+    def bwd(k):
+        i, o = batches[k % len(batches)]
+        dq.dq_embbag_int4_bwd_sgd(mt, d, i, o, B, n_ids[k % len(batches)], grads[k % len(batches)], 0.05,
+                                  dq.DQ_MODE_GREEDY, ws, ws.numel(), None, stream)
+
+    bwd(0)
+    e0.record(stream)
+    K = 10
+    for k in range(K):
+        bwd(k)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    b_ms = e0.elapsed_time(e1)
+    ids = sum(n_ids[k % len(batches)] for k in range(K))
+    rows = sum(touched[k % len(batches)] for k in range(K))
+    out["bwd"] = {
+        "what": "bag backward + SGD on the binary32 tables + greedy re-quantization of the touched rows, "
+                "one call per lookup batch",
+        "ids_per_s": ids / (b_ms / 1e3), "touched_rows_per_s": rows / (b_ms / 1e3), "ms_per_call": b_ms / K,
+        "requant_alu_frac_over_call": rows * EVALS_PER_ROW * FLOPS_PER_ELEMENT_EVAL * d / (b_ms / 1e3) / 1e12
+        / (2 * FP32_LANES_PER_SM * sms * 1965e6 / 1e12)}
+    return out
 
 
 def run_lookup_only(args, wl: W.Workload) -> None:
@@ -753,6 +847,8 @@ def main(argv=None) -> None:
     ap.add_argument("--lookup-only", action="store_true",
                     help="time only the lookup, over random packed tables of the workload's sizes")
     ap.add_argument("--streams", type=int, default=4, help="streams the per-table quantize launches spread over")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the codebook and backward legs that follow the timed region")
     ap.add_argument("--codebook", action="store_true",
                     help="time the codebook (k-means) quantizer and its lookup on the workload's tables")
     ap.add_argument("--bwd", action="store_true",
