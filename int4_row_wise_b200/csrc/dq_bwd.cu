@@ -22,13 +22,14 @@
 //   radix_scan_kernel    passes of three kernels each: per-tile digit counts,
 //   radix_scatter_kernel their digit-major exclusive scan, and a stable scatter
 //                        (warp-striped tiles ranked with ballots, no atomics)
-//   bwd_window_kernel    one warp per window: stages the entries' gradient rows in
-//                        shared memory (cp.async, all in flight), sums each row's
-//                        part in binary64; lists every row that ends in the window
-//                        (with its G when the row lies wholly inside it); a row
-//                        crossing a window edge leaves a binary64 part
+//   bwd_window_kernel    blocks take chunks of up to 8 windows (one atomic for the
+//                        chunk's list slots); a warp sums whole windows, EPL elements
+//                        per lane, the gradient rows staged in shared memory by
+//                        cp.async in double-buffered 4 KB stages; it lists every row
+//                        that ends in the window (with its G when the row lies wholly
+//                        inside it); a row crossing a window edge leaves a binary64 part
 //   bwd_span_kernel      one warp per (spanning row, 32 elements): adds its parts in
-//                        window order
+//                        window order, 32 parts prefetched to shared memory at a time
 // Every loop is bounded by sizes known at launch; no kernel waits on another.
 #include "dq_internal.cuh"
 
