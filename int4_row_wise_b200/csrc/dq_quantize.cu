@@ -79,22 +79,32 @@ __device__ __forceinline__ float exact_code(float x, float lo, float s)
     return fminf(fmaxf(q, 0.0f), kLevels);
 }
 
+// The W lanes of the calling lane's row. Rows of one warp may take different branches
+// (the per-row fast path), so the row's reductions name only its own lanes.
+template <int W>
+__device__ __forceinline__ unsigned row_mask()
+{
+    return W >= 32 ? 0xffffffffu : (((1u << (W & 31)) - 1u) << ((threadIdx.x & 31) & ~(W - 1)));
+}
+
 template <int W>
 __device__ __forceinline__ float row_sum(float v)
 {
+    const unsigned mask = row_mask<W>();
 #pragma unroll
     for (int o = 1; o < W; o <<= 1)
-        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+        v = __fadd_rn(v, __shfl_xor_sync(mask, v, o));
     return v;
 }
 
 template <int W>
 __device__ __forceinline__ void row_minmax(float &mn, float &mx)
 {
+    const unsigned mask = row_mask<W>();
 #pragma unroll
     for (int o = 1; o < W; o <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(mask, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(mask, mx, o));
     }
 }
 
@@ -389,23 +399,32 @@ __device__ __forceinline__ void quantize_one(const Row &src, const int d, const 
 
     const float range = __fsub_rn(mx, mn);
     const float step = __fdiv_rn(range, kSteps);
+    // Fast path, decided once per row. Every candidate has |lo| <= max(|xmin|, |xmax|)
+    // and width > 30 * step (the walk stops at 32 steps; when K <= 2^16 the grid
+    // points' rounding costs less than 0.25 step), so K bounds |lo * rcp(hi - lo)|
+    // for the whole walk, the starting clip included, and sets the tie margin.
+    const float w_min = __fmul_rn(step, 30.0f);
+    const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
+    const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
+    const TieWindow tw = tie_window(K);
     float lbest;
     {
+        // the starting clip (0, 0): grid points lo(0) = fma(0, step, xmin), hi(0) = fma(-0, step, xmax)
         float2 C0[H];
-        errors_exact<H, HAS_Y, FULL>(xp, mn, mx, kbase, d, C0);
+        if (fast) {
+            const Clip c0 = clip_fast(__fmaf_rn(0.0f, step, mn), __fmaf_rn(-0.0f, step, mx), tw);
+            bool hard = false;
+            errors_packed<H, HAS_Y, FULL>(xp, c0, kbase, d, C0, hard);
+            if (hard)
+                errors_fixup<H, HAS_Y, FULL>(xp, c0, kbase, d, C0);
+        } else {
+            errors_exact<H, HAS_Y, FULL>(xp, mn, mx, kbase, d, C0);
+        }
         lbest = row_sum<W>(tree_sum2<H>(C0));
     }
     float fbi = 0.0f, fbj = 0.0f;
     // A constant row has loss 0 at every grid point: the walk cannot change (0, 0).
     if (greedy && range != 0.0f) {
-        // Fast path, decided once per row. Every candidate has |lo| <= max(|xmin|, |xmax|)
-        // and width > 30 * step (the walk stops at 32 steps; when K <= 2^16 the grid
-        // points' rounding costs less than 0.25 step), so K bounds |lo * rcp(hi - lo)|
-        // for the whole walk and sets the tie margin.
-        const float w_min = __fmul_rn(step, 30.0f);
-        const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
-        const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
-        const TieWindow tw = tie_window(K);
         if (fast)
             greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
         else
