@@ -79,32 +79,24 @@ __device__ __forceinline__ float exact_code(float x, float lo, float s)
     return fminf(fmaxf(q, 0.0f), kLevels);
 }
 
-// The W lanes of the calling lane's row. Rows of one warp may take different branches
-// (the per-row fast path), so the row's reductions name only its own lanes.
-template <int W>
-__device__ __forceinline__ unsigned row_mask()
-{
-    return W >= 32 ? 0xffffffffu : (((1u << (W & 31)) - 1u) << ((threadIdx.x & 31) & ~(W - 1)));
-}
-
+// Sum over the W lanes of a row (the whole warp takes every shuffle: the walk's path
+// is chosen per warp, see quantize_one).
 template <int W>
 __device__ __forceinline__ float row_sum(float v)
 {
-    const unsigned mask = row_mask<W>();
 #pragma unroll
     for (int o = 1; o < W; o <<= 1)
-        v = __fadd_rn(v, __shfl_xor_sync(mask, v, o));
+        v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
 template <int W>
 __device__ __forceinline__ void row_minmax(float &mn, float &mx)
 {
-    const unsigned mask = row_mask<W>();
 #pragma unroll
     for (int o = 1; o < W; o <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(mask, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(mask, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
 }
 
@@ -405,13 +397,13 @@ __device__ __forceinline__ void quantize_one(const Row &src, const int d, const 
     // for the whole walk, the starting clip included, and sets the tie margin.
     const float w_min = __fmul_rn(step, 30.0f);
     const float K = __fmul_rn(fmaxf(fabsf(mn), fabsf(mx)), rcp_approx(w_min));
-    const bool fast = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
+    const bool fast_row = range <= kFastWMax && w_min >= kFastWMin && K <= kFastLoR;
     const TieWindow tw = tie_window(K);
     float lbest;
     {
         // the starting clip (0, 0): grid points lo(0) = fma(0, step, xmin), hi(0) = fma(-0, step, xmax)
         float2 C0[H];
-        if (fast) {
+        if (fast_row) {
             const Clip c0 = clip_fast(__fmaf_rn(0.0f, step, mn), __fmaf_rn(-0.0f, step, mx), tw);
             bool hard = false;
             errors_packed<H, HAS_Y, FULL>(xp, c0, kbase, d, C0, hard);
@@ -424,11 +416,30 @@ __device__ __forceinline__ void quantize_one(const Row &src, const int d, const 
     }
     float fbi = 0.0f, fbj = 0.0f;
     // A constant row has loss 0 at every grid point: the walk cannot change (0, 0).
-    if (greedy && range != 0.0f) {
+    const bool walk_row = greedy && range != 0.0f;
+    if constexpr (W == 1) {
+        // one row per lane: the walk has no shuffles, each row takes its own path
+        if (walk_row) {
+            if (fast_row)
+                greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
+            else
+                greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
+        }
+    } else if (__any_sync(0xffffffffu, walk_row)) {
+        // the walk's row shuffles run on the whole warp: the warp walks if any of its rows
+        // does (the others keep (0, 0)) and takes the fast path when every walking row
+        // qualifies; the two paths give identical losses
+        const bool fast = __all_sync(0xffffffffu, !walk_row || fast_row);
+        float lb = lbest, bi = 0.0f, bj = 0.0f;
         if (fast)
-            greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
+            greedy_walk<H, HAS_Y, FULL, true, W>(xp, kbase, d, mn, mx, step, tw, lb, bi, bj);
         else
-            greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, tw, lbest, fbi, fbj);
+            greedy_walk<H, HAS_Y, FULL, false, W>(xp, kbase, d, mn, mx, step, tw, lb, bi, bj);
+        if (walk_row) {
+            lbest = lb;
+            fbi = bi;
+            fbj = bj;
+        }
     }
     const int bi = (int)fbi, bj = (int)fbj;
 
