@@ -44,7 +44,9 @@ def compare_quant(g, o, d):
     oc = oc[:, :(d + 1) // 2]
     same = (np.all(gc == oc, axis=1) & np.all(gs == os_, axis=1) & np.all(gi == oi, axis=1)
             & (gl.view(np.uint32) == ol.view(np.uint32)))
-    rel = np.abs(gl.astype(np.float64) - ol) / np.maximum(np.abs(ol.astype(np.float64)), 1e-300)
+    with np.errstate(invalid="ignore"):  # inf - inf on rows whose loss overflows on both sides
+        rel = np.abs(gl.astype(np.float64) - ol) / np.maximum(np.abs(ol.astype(np.float64)), 1e-300)
+    rel[np.isnan(rel)] = 0
     rel[(gl == 0) & (ol == 0)] = 0
     return same, float(rel.max()) if rel.size else 0.0
 

@@ -141,3 +141,23 @@ def _tie_rows(n, d, seed):
 def test_rows_built_on_rounding_ties(cuda_device, d):
     x = _tie_rows(800 if d == 16 else 200, d, d)
     assert_quant_parity(x)
+
+
+@pytest.mark.parametrize("d", [32, 64, 128, 256])
+@pytest.mark.parametrize("mode", [dq.DQ_MODE_GREEDY, dq.DQ_MODE_MINMAX])
+def test_rows_of_one_warp_on_different_paths(cuda_device, d, mode):
+    # rows that share a warp (d >= 32) but need different walks: normal rows next to
+    # constant rows (no walk), rows outside the fast path's range (IEEE walk: huge range,
+    # offset far above the range, subnormal values), in every group of consecutive rows
+    r = np.random.default_rng(d)
+    specials = [
+        lambda: np.full(d, 2.5, np.float32),
+        lambda: np.linspace(-1e30, 1e30, d).astype(np.float32),
+        lambda: (1000.0 + 1e-3 * r.standard_normal(d)).astype(np.float32),
+        lambda: np.where(np.arange(d) % 2, 1e-39, 3e-39).astype(np.float32),
+        lambda: np.zeros(d, np.float32),
+    ]
+    rows = []
+    for i in range(600):
+        rows.append(specials[(i // 3) % len(specials)]() if i % 3 == 1 else r.standard_normal(d).astype(np.float32))
+    assert_quant_parity(np.stack(rows), mode=mode)
