@@ -84,6 +84,54 @@ __device__ __forceinline__ void nearest_all(const float (&x)[M], const float *c,
     }
 }
 
+// Same result as nearest_all when the 16 centroids are finite and non-decreasing:
+// fl(x - c) is monotone in c, so |fl(x - c_j)| does not rise while c_j <= x and does not
+// fall after it; the first minimum is the last c_j <= x (moved left over equal
+// distances) or the centroid after it. Four probes of a binary search find that c_j.
+template <int M>
+__device__ __forceinline__ void nearest_sorted(const float (&x)[M], const float *c, uint8_t (&q)[M])
+{
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        int cnt = 0;  // number of c_j <= x
+#pragma unroll
+        for (int step = 8; step >= 1; step >>= 1)
+            cnt = c[cnt + step - 1] <= x[m] ? cnt + step : cnt;
+        int j = 0;
+        if (cnt > 0) {
+            j = cnt - 1;
+            const float dl = fabsf(__fsub_rn(x[m], c[j]));
+            const bool right = j < 15 && fabsf(__fsub_rn(x[m], c[j + 1])) < dl;
+            if (right) {
+                j += 1;
+            } else {
+                while (j > 0 && fabsf(__fsub_rn(x[m], c[j - 1])) == dl)
+                    --j;
+            }
+        }
+        q[m] = (uint8_t)j;
+    }
+}
+
+// Are the row's centroids finite and non-decreasing (the condition of nearest_sorted)?
+__device__ __forceinline__ bool sorted_finite(const float *c)
+{
+    bool ok = isfinite(c[0]);
+#pragma unroll
+    for (int j = 1; j < 16; ++j)
+        ok &= isfinite(c[j]) && c[j - 1] <= c[j];
+    return ok;
+}
+
+template <int M>
+__device__ __forceinline__ void nearest(const float (&x)[M], const float *c, uint8_t (&q)[M])
+{
+    if (sorted_finite(c))
+        nearest_sorted<M>(x, c, q);
+    else
+        nearest_all<M>(x, c, q);
+}
+
 // One row per W lanes, M contiguous elements per lane; FULL: d == M * W.
 template <int M, int W, bool FULL>
 __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
@@ -116,7 +164,7 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
     }
     // the row's 16 centroids live in shared memory (every lane of the row writes the
     // same values; __syncwarp orders the writes before the reads)
-    __shared__ float cs_all[128 / W][16];
+    __shared__ float cs_all[128 / W][17];  // padded: rows' slots start in different banks
     float *c = cs_all[threadIdx.x / W];
     // K1: the min/max levels
     const float step = __fdiv_rn(__fsub_rn(mx, mn), kLevels);
@@ -129,7 +177,7 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
     // K2: Lloyd iterations
     uint8_t q[M];
     for (int it = 0; it < a.iters; ++it) {
-        nearest_all<M>(x, c, q);
+        nearest<M>(x, c, q);
         __syncwarp();  // every lane has read the centroids before they change
 #pragma unroll 1
         for (int j = 0; j < 16; ++j) {
@@ -158,7 +206,7 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
         }
     }
     __syncwarp();
-    nearest_all<M>(x, c, q);
+    nearest<M>(x, c, q);
     float e2[M];
 #pragma unroll
     for (int m = 0; m < M; ++m) {
