@@ -1,0 +1,124 @@
+"""Table-wise sharded lookup with the all-to-all of pooled outputs ("Deep Learning
+Recommendation Model for Personalization and Recommendation Systems", 提出的方法:
+model-parallel tables, data-parallel ranks), as gloo ranks on CPU: every rank's slice
+of the batch equals the single-process lookup over all tables, bit for bit. The
+per-rank lookup is the oracle's (this host has no GPU); on GPUs it is
+dq_embbag_int4_fwd and the exchange runs over NCCL."""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from int4_row_wise_b200.sharded import plan_tables, sharded_embbag
+
+D = 8
+
+
+def _problem(T, B, seed):
+    r = np.random.default_rng(seed)
+    rows = [int(n) for n in r.integers(0, 400, T)]
+    rows[0] = 0 if T > 3 else rows[0]  # an empty table when there are several
+    tables = []
+    for n in rows:
+        x = r.standard_normal((max(n, 1), D)).astype(np.float32)[:n]
+        c, sb, _, _ = oracle.quantize_rows(x) if n else (np.zeros((0, 4), np.uint8), np.zeros((0, 2), np.uint16),
+                                                          None, None)
+        tables.append((c, sb))
+    per_table = []
+    for t, n in enumerate(rows):
+        lens = r.integers(0, 5, B)
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        idx = r.integers(-2, max(n, 1) + 3, off[-1]).astype(np.int32)  # some ids out of range
+        per_table.append((idx, off))
+    return rows, tables, per_table
+
+
+def _batch_of(tables_sel, per_table):
+    """Table-major indices/offsets over the selected tables."""
+    idx, off = [], [0]
+    for t in tables_sel:
+        i, o = per_table[t]
+        idx.append(i)
+        off.extend((o[1:] + off[-1]).tolist())
+    return (np.concatenate(idx) if idx else np.zeros(0, np.int32)).astype(np.int32), np.array(off, np.int32)
+
+
+def _oracle_lookup(tables, d, indices, offsets, batch):
+    out, _, _ = oracle.embbag([(c, s) for c, s in tables], d, indices.numpy(), offsets.numpy(), batch)
+    return torch.from_numpy(out)
+
+
+def _rank(rank, world, port, T, B, seed, results):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rows, tables, per_table = _problem(T, B, seed)
+        owner = plan_tables(rows, world)
+        mine = [t for t in range(T) if owner[t] == rank]
+        idx, off = _batch_of(mine, per_table)
+        out = sharded_embbag([tables[t] for t in mine], owner, D, torch.from_numpy(idx), torch.from_numpy(off), B,
+                             lookup=_oracle_lookup)
+        results[rank] = out.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+@pytest.mark.parametrize("world,T,B,seed", [(2, 5, 6, 0), (3, 7, 9, 1), (3, 2, 3, 2), (2, 1, 4, 3)])
+def test_sharded_lookup_equals_the_single_device_lookup(world, T, B, seed):
+    rows, tables, per_table = _problem(T, B, seed)
+    idx, off = _batch_of(list(range(T)), per_table)
+    want = _oracle_lookup(tables, D, torch.from_numpy(idx), torch.from_numpy(off), B).numpy()
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_rank, args=(world, _free_port(), T, B, seed, results), nprocs=world, start_method="spawn")
+    bl = B // world
+    for r in range(world):
+        assert np.array_equal(results[r].view(np.uint32), want[r * bl:(r + 1) * bl].view(np.uint32)), r
+
+
+def test_plan_is_deterministic_and_balanced():
+    r = np.random.default_rng(5)
+    for world in (1, 2, 3, 8):
+        rows = [int(n) for n in r.integers(1, 10 ** 6, 26)]
+        a, b = plan_tables(rows, world), plan_tables(rows, world)
+        assert a == b and set(a) <= set(range(world))
+        load = [sum(n for n, o in zip(rows, a) if o == k) for k in range(world)]
+        assert max(load) - min(load) <= max(rows)
+    assert plan_tables([5, 5, 5], 2) == [0, 1, 0]  # equal loads go to the lower rank
+
+
+@pytest.mark.gpu
+def test_sharded_lookup_on_the_gpu_one_rank(cuda_device):
+    # the default path on a B200: dq_embbag_int4_fwd per rank and the exchange over NCCL
+    # (one rank here: every run of this build has one GPU)
+    import int4_row_wise_b200 as dq
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    import datetime
+    dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", 0))
+    try:
+        T, B = 4, 64
+        rows, tables, per_table = _problem(T, B, 7)
+        owner = plan_tables(rows, 1)
+        idx, off = _batch_of(list(range(T)), per_table)
+        dt = [dq.PackedTable(torch.from_numpy(np.ascontiguousarray(c)).cuda(),
+                             torch.from_numpy(np.ascontiguousarray(s).view(np.int16)).cuda()) for c, s in tables]
+        got = sharded_embbag(dt, owner, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
+        want = dq.embbag(dt, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
+        torch.cuda.synchronize()
+        assert torch.equal(got.view(torch.int32), want.view(torch.int32))
+    finally:
+        dist.destroy_process_group()
