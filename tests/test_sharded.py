@@ -118,7 +118,56 @@ def test_sharded_lookup_on_the_gpu_one_rank(cuda_device):
                              torch.from_numpy(np.ascontiguousarray(s).view(np.int16)).cuda()) for c, s in tables]
         got = sharded_embbag(dt, owner, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
         want = dq.embbag(dt, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
+        from int4_row_wise_b200.sharded import sharded_embbag_local
+        routed = sharded_embbag_local(dt, owner, D, [(torch.from_numpy(i).cuda(), torch.from_numpy(o).cuda())
+                                                     for i, o in per_table], B)
         torch.cuda.synchronize()
         assert torch.equal(got.view(torch.int32), want.view(torch.int32))
+        assert torch.equal(routed.view(torch.int32), want.view(torch.int32))
     finally:
         dist.destroy_process_group()
+
+
+def _local_problem(T, bl, rank, seed):
+    """This rank's own bags for every table (its local samples)."""
+    r = np.random.default_rng(seed * 1000 + rank)
+    rows, tables, _ = _problem(T, 1, seed)
+    batches = []
+    for n in rows:
+        lens = r.integers(0, 5, bl)
+        off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        idx = r.integers(-1, max(n, 1) + 2, off[-1]).astype(np.int32)
+        batches.append((idx, off))
+    return rows, tables, batches
+
+
+def _rank_local(rank, world, port, T, bl, seed, results):
+    from int4_row_wise_b200.sharded import sharded_embbag_local
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rows, tables, batches = _local_problem(T, bl, rank, seed)
+        owner = plan_tables(rows, world)
+        mine = [t for t in range(T) if owner[t] == rank]
+        out = sharded_embbag_local([tables[t] for t in mine], owner, D,
+                                   [(torch.from_numpy(i), torch.from_numpy(o)) for i, o in batches], bl,
+                                   lookup=_oracle_lookup)
+        results[rank] = out.numpy().copy()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,T,bl,seed", [(2, 5, 3, 0), (3, 6, 4, 1), (3, 2, 2, 2)])
+def test_routed_lookup_from_local_batches(world, T, bl, seed):
+    # every rank starts with its own samples' bags for all tables; the ids travel to the
+    # owners and the pooled rows back: each rank gets the single-device lookup of its bags
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_rank_local, args=(world, _free_port(), T, bl, seed, results), nprocs=world,
+                       start_method="spawn")
+    for r in range(world):
+        rows, tables, batches = _local_problem(T, bl, r, seed)
+        idx, off = _batch_of(list(range(T)), batches)
+        want = _oracle_lookup(tables, D, torch.from_numpy(idx), torch.from_numpy(off), bl).numpy()
+        assert np.array_equal(results[r].view(np.uint32), want.view(np.uint32)), r
