@@ -32,7 +32,8 @@
  * Conventions for every entry point:
  *   - All data pointers are DEVICE pointers (except `tables`, a host array). The
  *     caller owns every buffer; the library allocates no memory and keeps no
- *     state besides cached device attributes.
+ *     state besides cached device attributes (and, for
+ *     dq_embbag_int4_bwd_sgd_noalloc, its static device scratch array).
  *   - Calls are asynchronous and stream-ordered on `cuda_stream` (a cudaStream_t;
  *     NULL = the legacy default stream). Outputs are valid after the stream is
  *     synchronized. Calls may be made from several host threads.
