@@ -14,6 +14,13 @@ data path; timing is the max over ranks (weak scaling).
 
 --impl reference times the CPU oracle on the same workload (a bounded sample of
 rows per step, extrapolated to the whole step), on rank 0 only.
+
+After the timed region the line also reports, on rank 0: the pages' quality measure
+(`quality`, `l2_eval`), the codebook quantizer and the bag backward + SGD +
+re-quantization on the step's own tables (`next_rows`; --no-next-rows skips them),
+the end-to-end leg from pinned host memory (`e2e`) and the CPU oracle (`cpu_baseline`).
+Other modes, one JSON line each: --lookup-only (the lookup alone), --bwd (the bag
+backward + SGD + re-quantization), --codebook (the codebook quantizer and its lookup).
 """
 from __future__ import annotations
 
