@@ -224,7 +224,6 @@ def dequantize_rows_kmeans(codes: np.ndarray, codebook: np.ndarray, d: int) -> n
     return out
 
 
-BWD_WINDOW = 64
 BAD_OFFSETS = -2
 
 

@@ -55,12 +55,13 @@
  *      the number of indices; otherwise nothing changes. Every position p of bag
  *      (t, b) with a valid id gives an entry (key = row_base[t] + id, p), row_base[t]
  *      = rows of the tables before t. Invalid ids give no entry.
- *   b. The entries are sorted by (key, p). Their list is cut into windows of 64
- *      consecutive entries (positions 0..63, 64..127, ...).
- *   c. Gradient of a row, element k: the binary64 sum, from +0 in list order, of
- *      g[b][t*d + k] over the row's entries inside each window; these window parts
- *      are added, from +0 in window order, in binary64; G_k is that total rounded
- *      once to binary32.
+ *   b. The entries are sorted by (key, p), so each row's entries are together, in
+ *      the order of their positions in `indices`.
+ *   c. Gradient of a row, element k: the plain binary64 sum, from +0, of
+ *      g[b][t*d + k] over the row's entries in that order (one addition after the
+ *      other), rounded once to binary32 (G_k). Any order gives a valid sum; this is
+ *      the plainest one, and the CUDA path is compared with it within a stated
+ *      tolerance rather than required to share its order.
  *   d. W[id][k] = fma(-lr, G_k, W[id][k]) (binary32, rounded once).
  *   e. Each touched row (one with at least one entry) is quantized again from its new
  *      master values by the quantizer above (greedy or min/max); other rows keep
@@ -622,8 +623,6 @@ static void *bag_worker(void *arg)
     return NULL;
 }
 
-#define ORACLE_BWD_WINDOW 64
-
 typedef struct {
     uint32_t key;
     int32_t bag;
@@ -696,7 +695,6 @@ int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *con
     }
     /* b. sort by (key, p) */
     qsort(e, (size_t)ne, sizeof(bwd_entry), entry_cmp);
-    double *part = (double *)malloc(sizeof(double) * (size_t)d);
     double *sum = (double *)malloc(sizeof(double) * (size_t)d);
     float cbuf[ORACLE_MAX_D];
     for (int64_t s0 = 0; s0 < ne;) {
@@ -704,31 +702,21 @@ int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *con
         while (s1 < ne && e[s1].key == e[s0].key)
             s1++;
         if (sample_keys && !in_sample(sample_keys, n_sample, e[s0].key)) {
-            s0 = s1;  /* steps c-e only for the sampled rows (the windows still count every entry) */
+            s0 = s1;  /* steps c-e only for the sampled rows */
             continue;
         }
         int t = 0;
         while (t + 1 < T && (int64_t)e[s0].key >= row_base[t + 1])
             t++;
         int64_t id = (int64_t)e[s0].key - row_base[t];
-        /* c. window parts, then their sum */
+        /* c. the row's gradient: one binary64 sum over its entries, in list order */
         for (int k = 0; k < d; k++)
             sum[k] = 0.0;
-        for (int64_t w0 = s0; w0 < s1;) {
-            int64_t w1 = (w0 / ORACLE_BWD_WINDOW + 1) * ORACLE_BWD_WINDOW;
-            if (w1 > s1)
-                w1 = s1;
+        for (int64_t i = s0; i < s1; i++) {
+            int64_t b = e[i].bag - (int64_t)t * B;
+            const float *gr = grad + b * (int64_t)T * d + (int64_t)t * d;
             for (int k = 0; k < d; k++)
-                part[k] = 0.0;
-            for (int64_t i = w0; i < w1; i++) {
-                int64_t b = e[i].bag - (int64_t)t * B;
-                const float *gr = grad + b * (int64_t)T * d + (int64_t)t * d;
-                for (int k = 0; k < d; k++)
-                    part[k] = part[k] + (double)gr[k];
-            }
-            for (int k = 0; k < d; k++)
-                sum[k] = sum[k] + part[k];
-            w0 = w1;
+                sum[k] = sum[k] + (double)gr[k];
         }
         /* d. SGD step */
         float *w = W[t] + id * w_ld[t];
@@ -739,7 +727,6 @@ int64_t oracle_embbag_bwd_sgd(float *const *W, const int64_t *w_ld, uint8_t *con
         finish_row(w, d, &r, codes[t] + id * codes_ld[t], scale_bias[t] + 2 * id);
         s0 = s1;
     }
-    free(part);
     free(sum);
     free(e);
     free(row_base);

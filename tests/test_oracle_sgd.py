@@ -3,9 +3,9 @@
 Reading (the DQRM repository page trains INT4 embedding tables with quantization-
 aware training on binary32 masters; the pages fix no arithmetic for the step):
 entries (key = row_base[t] + id, position p) sorted by (key, p); a row's gradient is
-summed in binary64 inside windows of 64 consecutive entries of that sorted list,
-then across windows, and rounded once to binary32 (G); the master becomes
-fma(-lr, G, w); every touched row is quantized again.
+the plain binary64 sum of its entries' output-gradient rows, from +0, one addition
+after the other in that list order, rounded once to binary32 (G); the master
+becomes fma(-lr, G, w); every touched row is quantized again.
 """
 from fractions import Fraction
 
@@ -43,7 +43,7 @@ def _bags(T, B, n, lo, hi, seed):
 
 def _dyadic_grad(B, cols, seed):
     # k * 2^-40 with |k| < 2^44: every binary64 sum of a few hundred of them is exact,
-    # so the window order cannot matter and G is the exact sum rounded once.
+    # so no summation order can matter and G is the exact sum rounded once.
     r = np.random.default_rng(seed)
     k = r.integers(-(1 << 20), 1 << 20, (B, cols)).astype(np.float64)
     e = r.integers(-40, -16, (B, cols)).astype(np.float64)
@@ -87,18 +87,15 @@ def test_sgd_is_exact_gradient_then_one_fma(lr):
         assert np.array_equal(C[t][rows], c) and np.array_equal(S[t][rows], sb)
 
 
-def _window_case(prefix, tiny_at):
-    """One table, one-hot bags; `prefix` bags of row 0 come first, then 67 bags of row 1
-    whose gradients are 1, 2^-24, zeros, and 2^-54 at the entries listed in tiny_at
-    (entry numbers counted within row 1's run)."""
-    n_b = prefix + 67
-    idx = np.array([0] * prefix + [1] * 67, np.int32)
+def _one_row_case(prefix, row_grads):
+    """One table, one-hot bags: `prefix` bags of row 0 come first, then one bag of row 1
+    per value in row_grads (its output gradient, d = 1). W = 0 and lr = 1, so row 1's
+    new master is -G."""
+    n_b = prefix + len(row_grads)
+    idx = np.array([0] * prefix + [1] * len(row_grads), np.int32)
     off = np.arange(n_b + 1, dtype=np.int32)
     g = np.zeros((n_b, 1), np.float32)
-    g[prefix + 0, 0] = 1.0
-    g[prefix + 1, 0] = 2.0 ** -24
-    for e in tiny_at:
-        g[prefix + e, 0] = 2.0 ** -54
+    g[prefix:, 0] = np.asarray(row_grads, np.float64).astype(np.float32)
     W = [np.zeros((2, 1), np.float32)]
     C = [np.zeros((2, 1), np.uint8)]
     S = [np.zeros((2, 2), np.uint16)]
@@ -106,22 +103,36 @@ def _window_case(prefix, tiny_at):
     return W[0][1, 0]
 
 
-def test_window_split_changes_the_rounding():
-    # Entries 64..66 of row 1 (sorted positions 64..66) fall in the second window, whose
-    # part 3 * 2^-54 lifts 1 + 2^-24 above the binary32 midpoint: G = 1 + 2^-23.
-    assert _window_case(0, [64, 65, 66]) == -(1 + 2.0 ** -23)
-    # Inside one window the sum is sequential: each 2^-54 is a quarter of an ulp and is
-    # lost, G = 1 + 2^-24 rounds to even, G = 1.
-    assert _window_case(0, [2, 3, 4]) == -1.0
+TINY = 2.0 ** -54  # a quarter of the binary64 ulp of 1
 
 
-def test_windows_are_aligned_on_the_whole_sorted_list():
-    # 32 entries of row 0 come first: row 1's entries 32..34 sit at sorted positions
-    # 64..66, the second window, so they are summed apart from the 1 and the 2^-24.
-    assert _window_case(32, [32, 33, 34]) == -(1 + 2.0 ** -23)
-    # (Windows cut at the row's own first entry would put entries 32..34 with the 1.)
-    # Entries 29..31 sit at positions 61..63, in the first window with the 1: G = 1.
-    assert _window_case(32, [29, 30, 31]) == -1.0
+@pytest.mark.parametrize("prefix", [0, 1, 32, 63])
+@pytest.mark.parametrize("tiny_at", [(2, 3, 4), (64, 65, 66), (30, 31, 32, 33)])
+def test_gradient_is_a_binary64_sum_not_the_exact_one(prefix, tiny_at):
+    # 1 then 2^-24 (the binary32 midpoint above 1, exact in binary64), then zeros and a
+    # few 2^-54 later on. One addition at a time in binary64, each 2^-54 falls below half
+    # an ulp of the running sum and is lost, wherever it sits in the list: G = 1 + 2^-24,
+    # a binary32 tie, rounds to even, G = 1. The exact sum lies above the midpoint and
+    # would round to 1 + 2^-23.
+    grads = [0.0] * 70
+    grads[0], grads[1] = 1.0, 2.0 ** -24
+    for e in tiny_at:
+        grads[e] = TINY
+    exact = Fraction(1) + Fraction(1, 2 ** 24) + len(tiny_at) * F(np.float64(TINY))
+    assert round_to_f32(exact) == 1 + 2.0 ** -23
+    assert _one_row_case(prefix, grads) == -1.0
+
+
+def test_gradient_is_summed_in_list_order():
+    # The same values, the 2^-54 first: 3 * 2^-54 is exact, 1 + 3 * 2^-54 rounds up to
+    # 1 + 2^-52 in binary64, adding 2^-24 is exact, and the binary32 rounding now goes
+    # up: G = 1 + 2^-23. Only the order of the entries in the list differs from the
+    # case above (a binary32 running sum would give 1 both ways).
+    assert _one_row_case(5, [TINY, TINY, TINY, 1.0, 2.0 ** -24]) == -(1 + 2.0 ** -23)
+    assert _one_row_case(5, [1.0, 2.0 ** -24, TINY, TINY, TINY]) == -1.0
+    # cancellation: 1 + 2^-60 loses the 2^-60 in binary64; after -1 it is 0
+    assert _one_row_case(0, [1.0, 2.0 ** -60, -1.0]) == 0.0
+    assert _one_row_case(0, [1.0, -1.0, 2.0 ** -60]) == -(2.0 ** -60)
 
 
 def test_invalid_ids_skip_duplicates_count_twice_and_tables_are_separate():
@@ -176,7 +187,7 @@ def test_min_max_mode_requantizes_with_min_max():
 
 def test_sample_updates_exactly_the_sampled_rows():
     # a sample restricts steps c-e to its rows; each sampled row gets what the full
-    # call gives it (the windows still count every entry)
+    # call gives it
     T, B, n, d = 2, 60, 40, 4
     W, C, S = _tables(T, n, d, 21)
     idx, off = _bags(T, B, n, 1, 9, 22)
