@@ -283,9 +283,13 @@ dq_status dq_embbag_int4_bwd_sgd(const dq_master_table *tables, int32_t n_tables
  * held by every GPU that loads the library until the process exits. The call
  * allocates nothing. Arguments and results are those of dq_embbag_int4_bwd_sgd; a
  * call whose dq_embbag_int4_bwd_workspace_bytes(d, n_indices) exceeds the array is
- * rejected with DQ_ERR_INVALID_ARG (about 110,000 entries at d = 64).
+ * rejected with DQ_ERR_INVALID_ARG (at most 378,856 entries at d = 16, 114,687 at
+ * d = 64, 59,427 at d = 128).
  * The first call on a device looks up the array's device address there (once per
- * device), so make it before any stream capture. All calls share the array: calls
+ * device), so make it before any stream capture. The address is cached per device
+ * ordinal for the life of the process: after a cudaDeviceReset of a device the cached
+ * address is stale, so do not call this entry point on that device again in the same
+ * process. All calls share the array: calls
  * whose work overlaps on the GPU (several streams or host threads) race and must be
  * serialized by the caller. Each call clears what must start at zero itself.
  */

@@ -8,7 +8,10 @@
 // In host code the array's name only stands in for the symbol; its device address
 // comes from cudaGetSymbolAddress, taken once per device (with that device
 // current) on the first call there. That first call should therefore come before
-// any stream capture. All calls share the array and it keeps the previous call's
+// any stream capture. The address is cached per device ordinal until the process
+// exits; a cudaDeviceReset recreates the device's context and module, after which
+// the cached address is stale (the header documents that such a device must not be
+// used with this entry point again). All calls share the array and it keeps the previous call's
 // contents: the backward clears the only part that must start at zero (its
 // 256-byte header) at the start of every call, and writes everything else before
 // reading it. Calls whose work overlaps on the GPU (other streams, other host
