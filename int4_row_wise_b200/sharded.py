@@ -7,8 +7,13 @@ rank through an all-to-all exchange).
 Each rank owns whole tables. For the global batch it looks up its own tables with
 dq_embbag_int4_fwd (or an injected lookup), then one all-to-all sends every rank
 the rows of its slice of the batch; each rank reassembles [batch / world, T * d] in
-table order, exactly what a single device computes for those bags. The exchange is
+table order, exactly what a single device computes for those bags. The exchanges are
 torch.distributed's all_to_all_single (NCCL between GPUs).
+
+Host synchronisation: sharded_embbag needs none; sharded_embbag_local reads two small
+count arrays back to the host (the all-to-all split sizes must be host integers):
+every table's first and last offset before the exchange, and the received per-(source,
+table) id counts after the bag lengths have been exchanged.
 """
 from __future__ import annotations
 
@@ -32,6 +37,35 @@ def plan_tables(rows: Sequence[int], world: int) -> List[int]:
     return owner
 
 
+def _check_owner(owner: Sequence[int], world: int) -> None:
+    if len(owner) == 0:
+        raise ValueError("no tables: the plan is empty")
+    bad = [r for r in owner if not 0 <= int(r) < world]
+    if bad:
+        raise ValueError(f"owner ranks {bad[:4]} outside [0, {world})")
+
+
+def _reassemble(recv, owner: Sequence[int], world: int, bl: int, d: int):
+    """[bl, T * d] in global table order from the received buffer, which holds, source
+    by source, [bl, tables of that source, d]. One concatenation kernel."""
+    import torch
+    T = len(owner)
+    counts = [0] * world
+    where = []                       # (source, slot within the source) of every global table
+    for t in range(T):
+        s = int(owner[t])
+        where.append((s, counts[s]))
+        counts[s] += 1
+    base, at = [], 0
+    for s in range(world):
+        base.append(at)
+        at += bl * counts[s] * d
+    chunks = {s: recv[base[s]:base[s] + bl * counts[s] * d].view(bl, counts[s], d)
+              for s in range(world) if counts[s]}
+    parts = [chunks[s][:, k:k + 1, :] for s, k in where]
+    return torch.cat(parts, dim=1).view(bl, T * d)
+
+
 def sharded_embbag(local_tables: Sequence, owner: Sequence[int], d: int, indices, offsets, global_batch: int,
                    group=None, lookup: Optional[Callable] = None):
     """Pooled outputs of this rank's slice of the global batch, over all tables.
@@ -50,11 +84,15 @@ def sharded_embbag(local_tables: Sequence, owner: Sequence[int], d: int, indices
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
+    _check_owner(owner, world)
     if global_batch % world:
         raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
     mine = [t for t, r in enumerate(owner) if r == rank]
     if len(mine) != len(local_tables):
         raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
+    if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
+        raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x {global_batch} bags "
+                         f"need {len(mine) * global_batch + 1}")
     if lookup is None:
         import int4_row_wise_b200 as dq
         lookup = dq.embbag
@@ -62,83 +100,81 @@ def sharded_embbag(local_tables: Sequence, owner: Sequence[int], d: int, indices
     bl = global_batch // world
     counts = [sum(1 for r in owner if r == s) for s in range(world)]
     if mine:
-        local = lookup(local_tables, d, indices, offsets, global_batch)       # [B, T_own * d]
-        dev, dt = local.device, local.dtype
-        send = local.reshape(world, bl, len(mine) * d).contiguous().reshape(-1)  # destination-major
+        # [world * bl, T_own * d], row-major: already destination-major (rank s gets rows s*bl ..)
+        send = lookup(local_tables, d, indices, offsets, global_batch).reshape(-1)
+        dev, dt = send.device, send.dtype
     else:  # a rank without tables still takes part in the exchange
         dev, dt = offsets.device, torch.float32
         send = torch.empty(0, dtype=dt, device=dev)
-    recv = torch.empty(bl * sum(counts) * d, dtype=dt, device=dev)
+    recv = torch.empty(bl * T * d, dtype=dt, device=dev)
     dist.all_to_all_single(recv, send, output_split_sizes=[bl * c * d for c in counts],
                            input_split_sizes=[bl * len(mine) * d] * world, group=group)
-    out = torch.empty((bl, T, d), dtype=dt, device=dev)
-    at = 0
-    for s in range(world):
-        if counts[s] == 0:
-            continue
-        chunk = recv[at:at + bl * counts[s] * d].view(bl, counts[s], d)
-        at += bl * counts[s] * d
-        out[:, [t for t, r in enumerate(owner) if r == s], :] = chunk
-    return out.view(bl, T * d)
+    return _reassemble(recv, owner, world, bl, d)
 
 
 def sharded_embbag_local(local_tables: Sequence, owner: Sequence[int], d: int, batches: Sequence, local_batch: int,
                          group=None, lookup: Optional[Callable] = None):
     """The whole hybrid-parallel lookup from data-parallel inputs: every rank holds the
     bags of its own `local_batch` samples for every table (`batches[t] = (indices,
-    offsets)`, CSR per table), and gets back [local_batch, T * d] for those samples.
+    offsets)`, offsets of length local_batch + 1, nondecreasing), and gets back
+    [local_batch, T * d] for those samples.
 
-    Steps: the bag lengths and the ids of every table travel to the table's owner (two
-    all-to-alls: per-destination id counts, then lengths and ids); each owner lays out
-    its tables' global batch in rank order (rank 0's bags first); sharded_embbag looks
-    them up and returns every rank its slice."""
+    Steps: the bag lengths of every table travel to the table's owner (fixed-size
+    all-to-all), then the ids (one all-to-all with the split sizes read back from the
+    lengths); each owner lays out its tables' global batch in rank order (rank 0's bags
+    first); sharded_embbag looks them up and returns every rank its slice."""
     import torch
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
+    _check_owner(owner, world)
     T = len(owner)
     if len(batches) != T:
         raise ValueError(f"{len(batches)} batches for {T} tables")
+    for t, (_, off) in enumerate(batches):
+        if int(off.numel()) != local_batch + 1:
+            raise ValueError(f"table {t}: offsets hold {int(off.numel())} entries, local_batch + 1 = "
+                             f"{local_batch + 1} expected")
     dev = batches[0][1].device
     to = [[t for t in range(T) if owner[t] == s] for s in range(world)]
     mine = to[rank]
-    # what this rank sends to s: the lengths of its bags for s's tables, then their ids
-    lens_out, ids_out, n_ids_out = [], [], []
+    dest_order = [t for s in range(world) for t in to[s]]          # tables by destination rank
+    # host read 1: first and last offset of every table (the ids each table sends)
+    offs = torch.stack([off.to(torch.int64) for _, off in batches])  # [T, local_batch + 1]
+    ends = offs[:, [0, -1]].cpu().tolist()
+    # the lengths, destination-major over tables
+    lens_all = (offs[:, 1:] - offs[:, :-1]).to(torch.int32)          # [T, local_batch]
+    lens_send = lens_all[torch.tensor(dest_order, device=dev)].reshape(-1)
+    ids_parts, n_ids_out = [], []
     for s in range(world):
-        ls, ids = [], []
+        n = 0
         for t in to[s]:
-            idx, off = batches[t]
-            ls.append((off[1:] - off[:-1]).to(torch.int32))
-            ids.append(idx[off[0]:off[-1]].to(torch.int32))
-        lens_out.append(torch.cat(ls) if ls else torch.empty(0, dtype=torch.int32, device=dev))
-        cat = torch.cat(ids) if ids else torch.empty(0, dtype=torch.int32, device=dev)
-        ids_out.append(cat)
-        n_ids_out.append(cat.numel())
-    # id counts per destination
-    cnt_send = torch.tensor(n_ids_out, dtype=torch.int64, device=dev)
-    cnt_recv = torch.empty(world, dtype=torch.int64, device=dev)
-    dist.all_to_all_single(cnt_recv, cnt_send, group=group)
-    n_ids_in = [int(v) for v in cnt_recv.tolist()]
-    # lengths: local_batch per table, fixed sizes
+            a, b = ends[t]
+            ids_parts.append(batches[t][0][a:b].to(torch.int32))
+            n += b - a
+        n_ids_out.append(n)
+    ids_send = torch.cat(ids_parts) if ids_parts else torch.empty(0, dtype=torch.int32, device=dev)
     lens_recv = torch.empty(world * local_batch * len(mine), dtype=torch.int32, device=dev)
-    dist.all_to_all_single(lens_recv, torch.cat(lens_out), output_split_sizes=[local_batch * len(mine)] * world,
+    dist.all_to_all_single(lens_recv, lens_send, output_split_sizes=[local_batch * len(mine)] * world,
                            input_split_sizes=[local_batch * len(to[s]) for s in range(world)], group=group)
+    lens = lens_recv.view(world, len(mine), local_batch)             # [source, table, bag]
+    # host read 2: ids per (source, table), which fixes the split sizes of the ids exchange
+    per_src_tab = lens.sum(dim=2).cpu().tolist()
+    n_ids_in = [int(sum(row)) for row in per_src_tab]
     ids_recv = torch.empty(sum(n_ids_in), dtype=torch.int32, device=dev)
-    dist.all_to_all_single(ids_recv, torch.cat(ids_out), output_split_sizes=n_ids_in,
-                           input_split_sizes=n_ids_out, group=group)
+    dist.all_to_all_single(ids_recv, ids_send, output_split_sizes=n_ids_in, input_split_sizes=n_ids_out,
+                           group=group)
     # the owner's batch, table-major over its tables, rank-major within a table
-    lens = lens_recv.view(world, len(mine), local_batch)           # [source, table, bag]
-    per_src_tab = lens.sum(dim=2).tolist()                         # ids per (source, table)
     src_base = [0]
     for s in range(world):
         src_base.append(src_base[-1] + n_ids_in[s])
-    ids_parts = []
+    parts = []
     for k in range(len(mine)):
         for s in range(world):
             start = src_base[s] + sum(per_src_tab[s][:k])
-            ids_parts.append(ids_recv[start:start + per_src_tab[s][k]])
-    indices = torch.cat(ids_parts) if ids_parts else torch.empty(0, dtype=torch.int32, device=dev)
+            parts.append(ids_recv[start:start + per_src_tab[s][k]])
+    indices = torch.cat(parts) if parts else torch.empty(0, dtype=torch.int32, device=dev)
     offsets = torch.zeros(len(mine) * world * local_batch + 1, dtype=torch.int32, device=dev)
     offsets[1:] = torch.cumsum(lens.permute(1, 0, 2).reshape(-1), dim=0).to(torch.int32)
     return sharded_embbag(local_tables, owner, d, indices, offsets, world * local_batch, group=group,

@@ -3,7 +3,8 @@ Recommendation Model for Personalization and Recommendation Systems", æå‡ºçš„æ
 model-parallel tables, data-parallel ranks), as gloo ranks on CPU: every rank's slice
 of the batch equals the single-process lookup over all tables, bit for bit. The
 per-rank lookup is the oracle's (this host has no GPU); on GPUs it is
-dq_embbag_int4_fwd and the exchange runs over NCCL."""
+dq_embbag_int4_fwd and the exchange runs over NCCL; the GPU tests compare that path with
+the oracle's lookup on the same packed tables."""
 import os
 import socket
 
@@ -19,19 +20,19 @@ from int4_row_wise_b200.sharded import plan_tables, sharded_embbag
 D = 8
 
 
-def _problem(T, B, seed):
+def _problem(T, B, seed, d=D, pool=(0, 4)):
     r = np.random.default_rng(seed)
     rows = [int(n) for n in r.integers(0, 400, T)]
     rows[0] = 0 if T > 3 else rows[0]  # an empty table when there are several
     tables = []
     for n in rows:
-        x = r.standard_normal((max(n, 1), D)).astype(np.float32)[:n]
-        c, sb, _, _ = oracle.quantize_rows(x) if n else (np.zeros((0, 4), np.uint8), np.zeros((0, 2), np.uint16),
-                                                          None, None)
+        x = r.standard_normal((max(n, 1), d)).astype(np.float32)[:n]
+        c, sb, _, _ = oracle.quantize_rows(x) if n else (np.zeros((0, (d + 1) // 2), np.uint8),
+                                                          np.zeros((0, 2), np.uint16), None, None)
         tables.append((c, sb))
     per_table = []
     for t, n in enumerate(rows):
-        lens = r.integers(0, 5, B)
+        lens = r.integers(pool[0], pool[1] + 1, B)
         off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
         idx = r.integers(-2, max(n, 1) + 3, off[-1]).astype(np.int32)  # some ids out of range
         per_table.append((idx, off))
@@ -99,31 +100,76 @@ def test_plan_is_deterministic_and_balanced():
     assert plan_tables([5, 5, 5], 2) == [0, 1, 0]  # equal loads go to the lower rank
 
 
-@pytest.mark.gpu
-def test_sharded_lookup_on_the_gpu_one_rank(cuda_device):
-    # the default path on a B200: dq_embbag_int4_fwd per rank and the exchange over NCCL
-    # (one rank here: every run of this build has one GPU)
-    import int4_row_wise_b200 as dq
+@pytest.fixture(scope="module")
+def nccl_one_rank(cuda_device):
+    """A one-rank NCCL process group on cuda:0 (every run of this build has one GPU)."""
+    import datetime
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(_free_port())
-    import datetime
     dist.init_process_group("nccl", rank=0, world_size=1, timeout=datetime.timedelta(seconds=60),
                             device_id=torch.device("cuda", 0))
+    yield
+    dist.destroy_process_group()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("d", [16, 64, 128])
+@pytest.mark.parametrize("pool", [(1, 1), (4, 12)])
+def test_sharded_lookup_on_the_gpu_against_the_oracle(nccl_one_rank, d, pool):
+    # the default path on a B200: dq_embbag_int4_fwd (the vectorised embbag_kernel at these
+    # widths, one-hot and pooled layouts) and the exchanges over NCCL, both from the global
+    # per-table batch and from the rank's own samples routed to the owners; compared with
+    # the oracle's lookup on the same packed tables, element by element within
+    # 1e-5 * sum|xhat| and bit for bit on bags of one id
+    import int4_row_wise_b200 as dq
+    from int4_row_wise_b200.sharded import sharded_embbag_local
+    from tests.gpu_util import bag_tolerance_check
+    T, B = 5, 256
+    rows, tables, per_table = _problem(T, B, 7 + d, d=d, pool=pool)
+    owner = plan_tables(rows, 1)
+    idx, off = _batch_of(list(range(T)), per_table)
+    cld = dq._codes_ld(d)
+    dt = []
+    for c, sb in tables:
+        cp = np.zeros((c.shape[0], cld), np.uint8)
+        cp[:, :c.shape[1]] = c
+        dt.append(dq.PackedTable(torch.from_numpy(cp).cuda(), torch.from_numpy(np.ascontiguousarray(sb).view(np.int16)).cuda()))
+    got = sharded_embbag(dt, owner, d, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
+    routed = sharded_embbag_local(dt, owner, d, [(torch.from_numpy(i).cuda(), torch.from_numpy(o).cuda())
+                                                 for i, o in per_table], B)
+    torch.cuda.synchronize()
+    ref, mag, _ = oracle.embbag(tables, d, idx, off, B, with_abs_sum=True)
+    lens = np.stack([o[1:] - o[:-1] for _, o in per_table], axis=1)          # [B, T]
+    one = np.repeat(lens == 1, d, axis=1)                                      # elements of one-id bags
+    for out in (got, routed):
+        o = out.cpu().numpy()
+        bag_tolerance_check(o, ref, mag)
+        assert np.array_equal(o[one].view(np.uint32), ref[one].view(np.uint32))
+
+
+def test_sharded_rejects_bad_shapes():
+    # a one-rank gloo group: the checks run before any collective
+    from int4_row_wise_b200.sharded import sharded_embbag_local
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(_free_port())
+    dist.init_process_group("gloo", rank=0, world_size=1)
     try:
-        T, B = 4, 64
-        rows, tables, per_table = _problem(T, B, 7)
+        rows, tables, per_table = _problem(3, 4, 0)
         owner = plan_tables(rows, 1)
-        idx, off = _batch_of(list(range(T)), per_table)
-        dt = [dq.PackedTable(torch.from_numpy(np.ascontiguousarray(c)).cuda(),
-                             torch.from_numpy(np.ascontiguousarray(s).view(np.int16)).cuda()) for c, s in tables]
-        got = sharded_embbag(dt, owner, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
-        want = dq.embbag(dt, D, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B)
-        from int4_row_wise_b200.sharded import sharded_embbag_local
-        routed = sharded_embbag_local(dt, owner, D, [(torch.from_numpy(i).cuda(), torch.from_numpy(o).cuda())
-                                                     for i, o in per_table], B)
-        torch.cuda.synchronize()
-        assert torch.equal(got.view(torch.int32), want.view(torch.int32))
-        assert torch.equal(routed.view(torch.int32), want.view(torch.int32))
+        bt = [(torch.from_numpy(i), torch.from_numpy(o)) for i, o in per_table]
+        with pytest.raises(ValueError, match="local_batch"):
+            sharded_embbag_local(tables, owner, D, bt, 5, lookup=_oracle_lookup)   # 4 bags, not 5
+        with pytest.raises(ValueError, match="no tables"):
+            sharded_embbag_local([], [], D, [], 4, lookup=_oracle_lookup)
+        with pytest.raises(ValueError, match="batches"):
+            sharded_embbag_local(tables, owner, D, bt[:2], 4, lookup=_oracle_lookup)
+        idx, off = _batch_of([0, 1, 2], per_table)
+        with pytest.raises(ValueError, match="offsets"):
+            sharded_embbag(tables, owner, D, torch.from_numpy(idx), torch.from_numpy(off[:-1]), 4,
+                           lookup=_oracle_lookup)
+        with pytest.raises(ValueError, match="owner ranks"):
+            sharded_embbag(tables, [0, 1, 0], D, torch.from_numpy(idx), torch.from_numpy(off), 4,
+                           lookup=_oracle_lookup)
     finally:
         dist.destroy_process_group()
 
