@@ -29,6 +29,7 @@ can be regenerated on its own, in any order and in any process.
 from __future__ import annotations
 
 import dataclasses
+import functools
 import math
 from typing import List, Optional, Tuple
 
@@ -94,6 +95,11 @@ def workload(name: str, seed: int = 0) -> Workload:
     return Workload(name, seed, d, (1_000_000,), "t3_outliers", 8192, (32, 32), None, False)
 
 
+def first_tables(wl: Workload, n: int) -> Workload:
+    """The workload restricted to its first n tables (same draws for those tables)."""
+    return dataclasses.replace(wl, rows=wl.rows[:max(1, n)])
+
+
 def table_block(wl: Workload, t: int, block: int) -> np.ndarray:
     """Rows [block*BLOCK_ROWS, min((block+1)*BLOCK_ROWS, n)) of table t, float32 [rows, d]."""
     n = wl.rows[t]
@@ -121,6 +127,50 @@ def table_block(wl: Workload, t: int, block: int) -> np.ndarray:
         x[hit, col] *= 50.0
         return x.astype(np.float32)
     raise ValueError(wl.values)
+
+
+def device_table(wl: Workload, t: int, device, rows_per_draw: int = 1 << 19):
+    """Table t drawn on a CUDA device with torch's generator: float32 [n, d].
+
+    For benches whose tables are too large to draw on the host in reasonable time
+    (the production-shaped workload holds 10.24G values). The distributions are those
+    of table_block; the random stream is torch's Philox keyed on (seed, workload,
+    table), so the values differ from the host draws of the same table. Student-t(3)
+    is drawn as z0 / sqrt((z1^2 + z2^2 + z3^2) / 3) from four standard normals."""
+    import torch
+    n, d = wl.rows[t], wl.d
+    key = np.random.SeedSequence([wl.seed, _WORKLOAD_KEYS[wl.name], t, _P_VALUES, 1 << 20]).generate_state(1)[0]
+    g = torch.Generator(device=device)
+    g.manual_seed(int(key))
+    out = torch.empty((n, d), dtype=torch.float32, device=device)
+
+    def t3(m):
+        z = torch.randn((4, m, d), generator=g, device=device)
+        return z[0] * torch.rsqrt(z[1:].square().sum(0) / 3.0)
+
+    for r0 in range(0, n, rows_per_draw):
+        m = min(rows_per_draw, n - r0)
+        o = out[r0:r0 + m]
+        if wl.values == "normal0.1":
+            torch.randn((m, d), generator=g, device=device, out=o).mul_(0.1)
+        elif wl.values == "normal0.05":
+            torch.randn((m, d), generator=g, device=device, out=o).mul_(0.05)
+        elif wl.values == "uniform_inv_sqrt_n":
+            a = 1.0 / math.sqrt(n)
+            torch.rand((m, d), generator=g, device=device, out=o).mul_(2 * a).sub_(a)
+        elif wl.values == "lognormal_t3":
+            scale = torch.randn((m, 1), generator=g, device=device).sub_(3.0).exp_()
+            o.copy_(t3(m) * scale)
+        elif wl.values == "t3_outliers":
+            scale = torch.randn((m, 1), generator=g, device=device).exp_()
+            x = t3(m) * scale
+            hit = torch.nonzero(torch.rand(m, generator=g, device=device) < 0.01).flatten()
+            col = torch.randint(0, d, (hit.numel(),), generator=g, device=device)
+            x[hit, col] *= 50.0
+            o.copy_(x)
+        else:
+            raise ValueError(wl.values)
+    return out
 
 
 def n_blocks(wl: Workload, t: int) -> int:
@@ -156,10 +206,20 @@ def sample_rows(wl: Workload, t: int, rows: np.ndarray) -> np.ndarray:
     return out
 
 
+@functools.lru_cache(maxsize=64)
 def _zipf_cdf(n: int, alpha: float) -> np.ndarray:
     w = np.arange(1, n + 1, dtype=np.float64) ** (-alpha)
     c = np.cumsum(w)
-    return c / c[-1]
+    c /= c[-1]
+    c.flags.writeable = False
+    return c
+
+
+@functools.lru_cache(maxsize=64)
+def _permutation(seed: int, wk: int, t: int, n: int) -> np.ndarray:
+    p = _rng(seed, wk, t, _P_PERM, 0).permutation(n)
+    p.flags.writeable = False
+    return p
 
 
 def lookup_batch(wl: Workload, batch_id: int = 0) -> Tuple[np.ndarray, np.ndarray]:
@@ -185,8 +245,7 @@ def lookup_batch(wl: Workload, batch_id: int = 0) -> Tuple[np.ndarray, np.ndarra
             v = np.searchsorted(_zipf_cdf(n, wl.zipf_alpha), r.random(m), side="right")
             v = np.minimum(v, n - 1)
             if wl.permute_ids:
-                perm = _rng(wl.seed, wk, t, _P_PERM, 0).permutation(n)
-                v = perm[v]
+                v = _permutation(wl.seed, wk, t, n)[v]
         lens.append(ln)
         ids.append(v)
     lens = np.concatenate(lens)
@@ -208,7 +267,7 @@ def random_packed_table(n_rows: int, d: int, seed: int, codes_ld: Optional[int] 
     cb = (d + 1) // 2
     codes_ld = cb if codes_ld is None else codes_ld
     r = _rng(seed, 99, n_rows, _P_PACKED, d)
-    raw = np.frombuffer(r.bytes(n_rows * cb), dtype=np.uint8).reshape(n_rows, cb)
+    raw = r.bit_generator.random_raw((n_rows * cb + 7) // 8).view(np.uint8)[:n_rows * cb].reshape(n_rows, cb)
     if codes_ld == cb:
         codes = raw.copy()
     else:
