@@ -142,8 +142,12 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
  *               sum over the bag of fma(q_k, scale, bias); an empty bag gives +0
  *   d_flags     device uint32 (nullable): DQ_FLAG_BAD_INDEX, DQ_FLAG_BAD_OFFSETS
  *
- * The sum is accumulated in binary32 in id order. A bag of one id returns that
- * row's dequantized values exactly.
+ * The sum is accumulated in binary32, and a bag of one id returns that row's
+ * dequantized values exactly. The order of the additions is not specified: when the
+ * bags average 4 ids or more, an id repeated among 32 consecutive positions of a bag
+ * is decoded once and added with its count as the weight of one fma, and partial
+ * sums over subsets of the bag's rows are added together at the end. Each output
+ * element stays within a few binary32 roundings per id of the exact sum.
  */
 dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d,
                              const int32_t *indices, const int32_t *offsets, int32_t batch,
@@ -247,7 +251,11 @@ size_t dq_embbag_int4_bwd_workspace_bytes(int32_t d, int64_t n_indices);
  *   4. Each touched row is quantized again from its new master values (as
  *      dq_quantize_rows_int4 with `mode`, without row_loss/best_ij); untouched rows
  *      keep their codes, scale/bias and master values.
- * The result does not depend on scheduling: repeated calls give identical bits.
+ * The result does not depend on scheduling: repeated calls give identical bits. Step 2
+ * is the binary64 sum of the row's entries in list order, associated differently: it
+ * equals that plain sum rounded once to binary32 except where the sum lies within
+ * binary64 rounding error of a binary32 rounding boundary (then the two differ by one
+ * ulp).
  *
  *   tables      HOST array of n_tables dq_master_table (1..DQ_MAX_TABLES)
  *   d           1..DQ_MAX_D

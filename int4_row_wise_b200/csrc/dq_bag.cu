@@ -102,17 +102,15 @@ __global__ void __launch_bounds__(256) dequant_generic_kernel(const DequantArgs 
 // ---------------------------------------------------------------------------
 // embedding bag
 //
-// A bag is handled by G = EG * IS lanes: EG = d / E element groups (E outputs,
-// E/2 code bytes per lane: one 8- or 16-byte load per row) times IS id strides
-// (lane `is` takes ids p0 + is, p0 + is + IS, ...). Lanes are numbered
-// eg * IS + is, so the IS partial sums of an element group sit in neighbouring
-// lanes; a shuffle reduce-scatter then leaves lane `is` holding E / IS finished
-// sums, contiguous in the output row, and the bag's row is written as one
-// contiguous run. Short bags (average pooling < 4, e.g. one-hot lookups) use
-// IS = 1 and many bags per warp for memory-level parallelism; their rows are
-// staged through shared memory so that each warp store covers whole rows. The
-// kernel reads the id count (the last offset) to pick the layout, so the host
-// need not know the pooling.
+// Two layouts in one kernel, chosen on the device from the id count (the last
+// offset), so the host need not know the pooling:
+//  - long bags (average pooling >= 4): one warp per bag; its ids are read 32 at a
+//    time (the first 32 one bag ahead), repeated ids merged, distinct rows spread
+//    over the warp's slots, partial sums added through shared memory;
+//  - short bags (one-hot lookups): a warp takes 32 bags, each lane writes 16-byte
+//    chunks of whole output rows straight from registers.
+// Either way a bag's sum is binary32 accumulation of the binary32 fma(q, s, b)
+// values, and a bag of one id returns its dequantized row exactly.
 // ---------------------------------------------------------------------------
 constexpr int kBagThreads = 256;
 
@@ -330,8 +328,8 @@ __device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagA
     }
 }
 
-// What a lane fetches ahead for one bag of the short-bag layout: its offsets and
-// the id at the bag's own position g (where a one-hot bag keeps its id).
+// What a lane fetches ahead for one bag of the one-hot layout: its offsets and the id
+// at the bag's own position g (where a one-hot bag keeps its id when every bag is).
 struct ShortAhead {
     int32_t p, p1, id;
 };
@@ -347,125 +345,239 @@ __device__ __forceinline__ ShortAhead short_ahead(const BagArgs &a, uint64_t g, 
     return s;
 }
 
-// The row of a one-hot bag whose id sits at its own position, loaded one tile ahead.
-template <int E>
-struct ShortRow {
-    typename CodeVec<E>::T w;
-    uint32_t sb;
-    bool ready;
+// The code bytes of EL elements (one lane's chunk of a row in the one-hot layout).
+template <int EL>
+struct ChunkVec;
+template <>
+struct ChunkVec<4> {
+    using T = uint16_t;
+    static __device__ __forceinline__ uint32_t word(const T &v, int) { return v; }
+};
+template <>
+struct ChunkVec<8> {
+    using T = uint32_t;
+    static __device__ __forceinline__ uint32_t word(const T &v, int) { return v; }
+};
+template <>
+struct ChunkVec<16> {
+    using T = uint2;
+    static __device__ __forceinline__ uint32_t word(const T &v, int i) { return i == 0 ? v.x : v.y; }
+};
+template <>
+struct ChunkVec<32> {
+    using T = uint4;
+    static __device__ __forceinline__ uint32_t word(const T &v, int i)
+    {
+        return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+    }
 };
 
-template <int E>
-__device__ __forceinline__ ShortRow<E> short_row(const BagTables &tabs, const BagArgs &a, const ShortAhead &s,
-                                                 uint64_t g, uint32_t total, int32_t n_ids, int eg)
+// The EL dequantized values fma(q, scale, bias) of a chunk, as EL / 4 float4.
+template <int EL>
+__device__ __forceinline__ void dequant_chunk_to(const typename ChunkVec<EL>::T &c, uint32_t sbw, float4 (&x)[EL / 4])
 {
-    ShortRow<E> r;
-    r.ready = false;
-    if (g < total && (int64_t)s.p == (int64_t)g && s.p1 == s.p + 1 && s.p1 <= n_ids) {
-        const int t = (int)div_batch((uint32_t)g, a.div);
-        const TableView tv = table_view(tabs, t, eg, E);
-        if ((uint32_t)s.id < tv.n_rows) {
-            r.w = __ldg(reinterpret_cast<const typename CodeVec<E>::T *>(tv.codes + (uint64_t)(uint32_t)s.id * tv.ld));
-            r.sb = __ldg(tv.sb + (uint32_t)s.id);
-            r.ready = true;
+    const float2 m23 = make_float2(-kTwo23, -kTwo23);
+    const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
+    const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
+    const float2 bb = make_float2(B, B);
+    const float2 s01 = make_float2(S, __fmul_rn(S, 0.0625f));
+    const float2 s23 = make_float2(__fmul_rn(S, 0.00390625f), __fmul_rn(S, 0.000244140625f));
+    if constexpr (EL == 4) {
+        const uint32_t w = ChunkVec<EL>::word(c, 0);
+        const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23), s01, bb);
+        const float2 x23 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23), s23, bb);
+        x[0] = make_float4(x01.x, x01.y, x23.x, x23.y);
+    } else {
+        const float S4 = __fmul_rn(S, 1.52587890625e-05f);
+        const float2 s42 = make_float2(S4, s23.x), s34 = make_float2(s23.y, S4);
+#pragma unroll
+        for (int i = 0; i < EL / 8; ++i) {
+            const uint32_t w = ChunkVec<EL>::word(c, i);
+            const uint32_t hi = w >> 12;
+            const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23), s01, bb);
+            const float2 x23 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23), s23, bb);
+            const float2 x45 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 4), magic_nibble(hi, 2)), m23), s42, bb);
+            const float2 x67 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(hi, 3), magic_nibble(hi, 4)), m23), s34, bb);
+            x[2 * i] = make_float4(x01.x, x01.y, x23.x, x23.y);
+            x[2 * i + 1] = make_float4(x45.x, x45.y, x67.x, x67.y);
         }
     }
-    return r;
 }
 
-// Short bags (one-hot lookups): many bags per warp, one lane per element group. A
-// two-stage pipeline keeps loads in flight across tiles: the offsets and the id at
-// the bag's own position two tiles ahead, the row of a one-hot bag one tile ahead.
-// Rows are staged in shared memory and written back as whole contiguous rows.
-template <int E>
-__device__ __forceinline__ void bag_tiles_short(const BagTables &tabs, const BagArgs &a, uint32_t total,
-                                                int32_t n_ids, float *stage)
+// Writes the EL dequantized values of a chunk as EL / 4 streaming float4 stores.
+template <int EL>
+__device__ __forceinline__ void dequant_chunk_store(const typename ChunkVec<EL>::T &c, uint32_t sbw, float4 *dst)
 {
-    const int EG = a.d / E;
-    const uint32_t bags_per_block = kBagThreads / EG;
-    const int lb = threadIdx.x / EG, eg = threadIdx.x % EG;
+    float4 x[EL / 4];
+    dequant_chunk_to<EL>(c, sbw, x);
+#pragma unroll
+    for (int k = 0; k < EL / 4; ++k)
+        __stcs(dst + k, x[k]);
+}
+
+// One bag of a warp's tile in the one-hot layout, in shared memory.
+struct OnehotSlot {
+    const uint8_t *code;   // the row's code bytes (kind 0)
+    const uint32_t *sb;    // the row's {scale, bias}
+    float *out;            // the bag's output row (nullptr past the last bag)
+    uint32_t kind;         // 0: one valid id; 1: zeros (empty bag, or one invalid id); 2: two or more ids
+    uint32_t pad;
+};
+
+// Short bags (average pooling < 4, e.g. one-hot lookups): a warp takes 32 consecutive
+// bags, one per lane for the bookkeeping (offsets, the id, the row and output
+// addresses, kept in a per-warp table in shared memory); the offsets and the id of the
+// next tile's bags are loaded one tile ahead. Then every lane produces one EL-element
+// chunk of a bag's output row per sub-step: LB = d / EL lanes cover a row, so a warp
+// store writes 32 / LB whole rows; the loads of UNR sub-steps are issued before any is
+// decoded, and a one-id bag's row is fma(q, scale, bias) written directly (no sum).
+// Bags with two or more ids are then summed one at a time by the warp's first LB lanes.
+template <int EL>
+__device__ __forceinline__ void bag_tiles_onehot(const BagTables &tabs, const BagArgs &a, uint32_t total,
+                                                 int32_t n_ids, OnehotSlot *slots)
+{
+    using CV = typename ChunkVec<EL>::T;
+    constexpr unsigned FULL = 0xffffffffu;
+    constexpr int UNR = EL >= 16 ? 4 : 8;         // sub-steps whose loads are in flight together
+    const int LB = a.d / EL;                      // lanes per row, a power of two <= 32
+    const int lb_bits = 31 - __clz(LB);
+    const int BPS = 32 >> lb_bits;                // bags per sub-step
     const int lane = threadIdx.x & 31;
-    const int bags_per_warp = 32 / EG;
-    const int q4_shift = 31 - __clz(a.d / 4);   // d / 4 float4 per row, a power of two
+    const int c = lane & (LB - 1);
+    const int bsub = lane >> lb_bits;
+    const uint64_t wpb = blockDim.x >> 5;
+    const uint64_t stride = (uint64_t)gridDim.x * wpb * 32;
     const uint32_t batch = (uint32_t)a.batch;
-    const uint64_t gstride = (uint64_t)gridDim.x * bags_per_block;
-    float *st = stage + (threadIdx.x >> 5) * 32 * (E + 4);
 
-    uint32_t tile = blockIdx.x;
-    const uint64_t g0 = (uint64_t)tile * bags_per_block + lb;
-    ShortAhead ahead1 = short_ahead(a, g0, total, n_ids);
-    ShortAhead ahead2 = short_ahead(a, g0 + gstride, total, n_ids);
-    ShortRow<E> row1 = short_row<E>(tabs, a, ahead1, g0, total, n_ids, eg);
-    for (; (uint64_t)tile * bags_per_block < total; tile += gridDim.x) {
-        const uint32_t g = tile * bags_per_block + lb;
-        const bool live = g < total;
-        const ShortAhead cur = ahead1;
-        const ShortRow<E> crow = row1;
-        ahead1 = ahead2;
-        ahead2 = short_ahead(a, (uint64_t)g + 2 * gstride, total, n_ids);
-        row1 = short_row<E>(tabs, a, ahead1, (uint64_t)g + gstride, total, n_ids, eg);
-
-        const int t = live ? (int)div_batch(g, a.div) : 0;
-        const int b = live ? (int)(g - (uint32_t)t * batch) : 0;
-        int32_t p = cur.p, p1 = cur.p1;
-        if (live)
-            clamp_bag(p, p1, n_ids, eg == 0, a.flags);
-        else
-            p = p1 = 0;
-        const TableView tv = table_view(tabs, t, eg, E);
-        float2 acc2[E / 2];
-#pragma unroll
-        for (int k = 0; k < E / 2; ++k)
-            acc2[k] = make_float2(0.0f, 0.0f);
-        bool bad = false;
-        if (crow.ready) {
-            accumulate_row<E>(crow.w, crow.sb, acc2);
-        } else if (p1 == p + 1) {
-            const uint32_t id = (uint32_t)__ldg(a.indices + p);
-            if (id < tv.n_rows)
-                accumulate_row<E>(__ldg(reinterpret_cast<const typename CodeVec<E>::T *>(tv.codes + (uint64_t)id * tv.ld)),
-                                  __ldg(tv.sb + id), acc2);
-            else
-                bad = true;
-        } else if (p1 > p) {
-            accumulate_ids<E>(a.indices, p, p1, 1, tv, acc2, bad);
-        }
-        if (bad)
-            raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
-
-        // stage the warp's rows (E + 4 floats per lane: conflict-free float4 writes)
-#pragma unroll
-        for (int k = 0; k < E / 2; k += 2)
-            *reinterpret_cast<float4 *>(st + lane * (E + 4) + 2 * k) =
-                make_float4(acc2[k].x, acc2[k].y, acc2[k + 1].x, acc2[k + 1].y);
-        __syncwarp();
-        // the warp's bags are consecutive: write each row as contiguous float4s; the
-        // first lane of each bag broadcasts its output row's address
-        float4 *row = reinterpret_cast<float4 *>(a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d);
-        const uint32_t gw = tile * bags_per_block + (uint32_t)((threadIdx.x >> 5) * bags_per_warp);
-        for (int f = lane; f < 8 * E; f += 32) {   // the warp's 32 * E / 4 float4
-            const int bw = f >> q4_shift, c = f & ((1 << q4_shift) - 1);
-            float4 *dst = reinterpret_cast<float4 *>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(row), bw * EG));
-            if (gw + bw < total) {
-                const int e0 = 4 * c;
-                dst[c] = *reinterpret_cast<const float4 *>(st + (bw * EG + e0 / E) * (E + 4) + (e0 % E));
+    uint64_t g0 = ((uint64_t)blockIdx.x * wpb + (threadIdx.x >> 5)) * 32;
+    ShortAhead nxt = short_ahead(a, g0 + lane, total, n_ids);
+    for (; g0 < total; g0 += stride) {
+        const ShortAhead cur = nxt;
+        nxt = short_ahead(a, g0 + stride + lane, total, n_ids);
+        const uint64_t g = g0 + lane;
+        OnehotSlot sl{nullptr, nullptr, nullptr, 1u, 0u};
+        if (g < total) {
+            int32_t p = cur.p, p1 = cur.p1;
+            clamp_bag(p, p1, n_ids, true, a.flags);
+            const int t = (int)div_batch((uint32_t)g, a.div);
+            const int b = (int)((uint32_t)g - (uint32_t)t * batch);
+            sl.out = a.out + ((int64_t)b * a.T + t) * a.d;
+            if (p1 == p + 1) {
+                const uint32_t id = (int64_t)p == (int64_t)g ? (uint32_t)cur.id : (uint32_t)__ldg(a.indices + p);
+                if ((int64_t)id < tabs.n_rows[t]) {
+                    sl.code = tabs.codes[t] + (uint64_t)id * (uint64_t)tabs.codes_ld[t];
+                    sl.sb = reinterpret_cast<const uint32_t *>(tabs.scale_bias[t]) + id;
+                    sl.kind = 0u;
+                } else {
+                    raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                }
+            } else if (p1 > p) {
+                sl.kind = 2u;
             }
         }
+        slots[lane] = sl;
         __syncwarp();
+        for (int s0 = 0; s0 < LB; s0 += UNR) {
+            CV w[UNR];
+            uint32_t sbw[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int s = s0 + u;
+                if (s < LB) {
+                    const OnehotSlot &q = slots[s * BPS + bsub];
+                    if (q.kind == 0u) {
+                        w[u] = __ldg(reinterpret_cast<const CV *>(q.code) + c);
+                        sbw[u] = __ldg(q.sb);
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int s = s0 + u;
+                if (s < LB) {
+                    const OnehotSlot &q = slots[s * BPS + bsub];
+                    float4 *dst = reinterpret_cast<float4 *>(q.out + c * EL);
+                    if (q.kind == 0u) {
+                        dequant_chunk_store<EL>(w[u], sbw[u], dst);
+                    } else if (q.kind == 1u && q.out != nullptr) {
+#pragma unroll
+                        for (int j = 0; j < EL / 4; ++j)
+                            __stcs(dst + j, make_float4(0.0f, 0.0f, 0.0f, 0.0f));
+                    }
+                }
+            }
+        }
+        // bags of two or more ids, one at a time: lanes 0..LB-1 sum their chunks in id order
+        uint32_t multi = __ballot_sync(FULL, sl.kind == 2u);
+        while (multi) {
+            const int j = __ffs(multi) - 1;
+            multi &= multi - 1;
+            const uint64_t gj = g0 + j;
+            int32_t p = __ldg(a.offsets + gj), p1 = __ldg(a.offsets + gj + 1);
+            clamp_bag(p, p1, n_ids, false, a.flags);
+            const int t = (int)div_batch((uint32_t)gj, a.div);
+            const TableView tv = table_view(tabs, t, 0, 0);
+            float acc[EL];
+#pragma unroll
+            for (int k = 0; k < EL; ++k)
+                acc[k] = 0.0f;
+            bool bad = false;
+            if (lane < LB) {
+                for (int32_t q0 = p; q0 < p1; q0 += 4) {   // four ids' rows in flight, added in id order
+                    uint32_t id[4];
+                    CV cw[4];
+                    uint32_t sbw[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        id[u] = q0 + u < p1 ? (uint32_t)__ldg(a.indices + q0 + u) : 0xffffffffu;
+                        if (id[u] < tv.n_rows) {
+                            cw[u] = __ldg(reinterpret_cast<const CV *>(tv.codes + (uint64_t)id[u] * tv.ld) + c);
+                            sbw[u] = __ldg(tv.sb + id[u]);
+                        } else if (q0 + u < p1) {
+                            bad = true;
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        if (id[u] >= tv.n_rows)
+                            continue;
+                        float4 x4[EL / 4];
+                        dequant_chunk_to<EL>(cw[u], sbw[u], x4);
+#pragma unroll
+                        for (int k = 0; k < EL / 4; ++k) {
+                            acc[4 * k] = __fadd_rn(acc[4 * k], x4[k].x);
+                            acc[4 * k + 1] = __fadd_rn(acc[4 * k + 1], x4[k].y);
+                            acc[4 * k + 2] = __fadd_rn(acc[4 * k + 2], x4[k].z);
+                            acc[4 * k + 3] = __fadd_rn(acc[4 * k + 3], x4[k].w);
+                        }
+                    }
+                }
+                float4 *dst = reinterpret_cast<float4 *>(slots[j].out + c * EL);
+#pragma unroll
+                for (int k = 0; k < EL / 4; ++k)
+                    dst[k] = make_float4(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3]);
+            }
+            if (__any_sync(FULL, bad) && lane == 0)
+                raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+        }
+        __syncwarp();   // the slots are rewritten by the next tile
     }
 }
 
-template <int E, int ISL>
+// E1: elements per lane chunk of the one-hot layout; E, ISL: elements per lane and
+// id strides of the long layout. The kernel reads the id count (the last offset) and
+// takes the long layout when bags average 4 ids or more.
+template <int E1, int E, int ISL>
 __global__ void __launch_bounds__(kBagThreads, E == 16 ? 4 : 1) embbag_kernel(const __grid_constant__ BagTables tabs,
-                                                             const BagArgs a)
+                                                                             const BagArgs a)
 {
-    __shared__ __align__(16) float stage[(kBagThreads / 32) * 32 * (E + 4)];
+    __shared__ __align__(16) OnehotSlot slots[kBagThreads / 32][32];
     const int64_t total = (int64_t)a.T * a.batch;
     const int32_t n_ids = max(__ldg(a.offsets + total), 0);
     if (ISL > 1 && (int64_t)n_ids >= 4 * total)   // average pooling >= 4: split ids over lanes
         bag_tiles_long<E, ISL>(tabs, a, (uint32_t)total, n_ids);
     else
-        bag_tiles_short<E>(tabs, a, (uint32_t)total, n_ids, stage);
+        bag_tiles_onehot<E1>(tabs, a, (uint32_t)total, n_ids, slots[threadIdx.x >> 5]);
 }
 
 // any d, any alignment: one warp per bag, lanes stride over the elements
@@ -550,18 +662,21 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, 
     if (fast) {
         const int EG = a.d / E;
         const int isl = EG <= 4 ? 8 : EG == 8 ? 4 : EG == 16 ? 2 : 1;
-        const int bags_per_block = kBagThreads / (EG * isl);
-        const int64_t tiles = (total + bags_per_block - 1) / bags_per_block;
+        const int64_t long_tiles = (total + kBagThreads / (EG * isl) - 1) / (kBagThreads / (EG * isl));
+        const int64_t onehot_blocks = (total + kBagThreads - 1) / kBagThreads;   // 32 bags per warp
+        const int64_t need = long_tiles > onehot_blocks ? long_tiles : onehot_blocks;
         const int64_t cap = (int64_t)num_sms * 8;
-        const unsigned grid = (unsigned)(tiles < cap ? tiles : cap);
-        if (E == 16) {
-            if (isl == 8) embbag_kernel<16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-            else if (isl == 4) embbag_kernel<16, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-            else if (isl == 2) embbag_kernel<16, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-            else embbag_kernel<16, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        } else {
-            embbag_kernel<32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);
-        }
+        const unsigned grid = (unsigned)(need < cap ? need : cap);
+        if (E == 32)
+            embbag_kernel<32, 32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);   // d = 1024
+        else if (isl == 8)
+            embbag_kernel<4, 16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 16, 32, 64
+        else if (isl == 4)
+            embbag_kernel<4, 16, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 128
+        else if (isl == 2)
+            embbag_kernel<8, 16, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 256
+        else
+            embbag_kernel<16, 16, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);   // d = 512
     } else {
         const int64_t grid = (total * 32 + 255) / 256;
         embbag_generic_kernel<<<(unsigned)grid, 256, 0, stream>>>(tabs, a);

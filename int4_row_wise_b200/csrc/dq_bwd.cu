@@ -13,7 +13,10 @@
 // row); the sorted list is cut into windows of 64 entries; a row's gradient is the
 // binary64 sum of its entries inside each window, then of those window parts in
 // window order, rounded once to binary32. The result is the same whatever the
-// scheduling, so the updated masters and their codes are reproducible.
+// scheduling, so the updated masters and their codes are reproducible. It is the
+// binary64 sum of the row's entries in list order, associated by windows: it can
+// differ from the plain sequential binary64 sum rounded once only where that sum lies
+// within binary64 rounding error of a binary32 rounding boundary (one ulp then).
 //
 // Kernels, in stream order:
 //   bwd_keys_kernel      one lane (or warp) per bag: writes (key, bag) of its entries;
