@@ -144,10 +144,9 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
  *
  * The sum is accumulated in binary32, and a bag of one id returns that row's
  * dequantized values exactly. The order of the additions is not specified: when the
- * bags average 4 ids or more, an id repeated among 32 consecutive positions of a bag
- * is decoded once and added with its count as the weight of one fma, and partial
- * sums over subsets of the bag's rows are added together at the end. Each output
- * element stays within a few binary32 roundings per id of the exact sum.
+ * bags average 4 ids or more, interleaved partial sums over the bag's ids are added
+ * together at the end. Each output element stays within a few binary32 roundings per
+ * id of the exact sum.
  */
 dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d,
                              const int32_t *indices, const int32_t *offsets, int32_t batch,
