@@ -6,13 +6,15 @@
 // Personalization and Recommendation Systems", section 提出的方法 (proposed
 // method), bullet 1, summed over each bag of ids.
 //
-// Both kernels are bound by HBM (and, for long bags, by integer/FP32 issue):
-// packed rows are read with 8- or 16-byte vector loads, outputs written with
-// 16-byte stores, and a nibble becomes a float with one LOP3 and one FADD:
-// OR-ing 0x4B000000 onto the nibble left in place at bits 4k..4k+3 gives the
-// float 2^23 + q*2^(4k); subtracting 2^23 leaves q*2^(4k) exactly, and an FMA
-// with scale*2^(-4k) (an exact power-of-two rescaling) gives fma(q, scale, bias)
-// bit for bit. Nibbles 5..7 of a word are shifted down by 12 bits first.
+// Both kernels are bound by HBM (and, for long bags, by instruction issue): packed
+// rows are read with 8- or 16-byte vector loads, outputs written with 16-byte stores.
+// A nibble becomes a float without integer-to-float conversion. The dequantize kernel
+// ORs 0x4B000000 onto the nibble left in place at bits 4k..4k+3 (the float
+// 2^23 + q*2^(4k); subtracting 2^23 leaves q*2^(4k) exactly, and an FMA with
+// scale*2^(-4k), an exact power-of-two rescaling, gives fma(q, scale, bias) bit for
+// bit). The lookup masks the even and odd nibbles into the low halves of bytes and
+// byte-permutes each under the exponent byte 0x4B (the float 2^23 + q), which takes
+// one instruction per element and one scale for all of them.
 #include "dq_internal.cuh"
 
 namespace dq {
@@ -130,45 +132,6 @@ struct CodeVec<32> {
     }
 };
 
-// scale * 2^(-4k) for the nibble pairs (0,1), (2,3), (4,5->2), (6->3,7->4) of a word
-struct PairParams {
-    float2 s01, s23, s42, s34, bb;
-};
-
-__device__ __forceinline__ PairParams pair_params(uint32_t sbw)
-{
-    const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
-    const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
-    const float S1 = __fmul_rn(S, 0.0625f), S2 = __fmul_rn(S, 0.00390625f);
-    const float S3 = __fmul_rn(S, 0.000244140625f), S4 = __fmul_rn(S, 1.52587890625e-05f);
-    PairParams p;
-    p.s01 = make_float2(S, S1);
-    p.s23 = make_float2(S2, S3);
-    p.s42 = make_float2(S4, S2);
-    p.s34 = make_float2(S3, S4);
-    p.bb = make_float2(B, B);
-    return p;
-}
-
-__device__ __forceinline__ float magic_nibble(uint32_t w, int k)
-{
-    return __uint_as_float((w & (0xfu << (4 * k))) | 0x4B000000u);
-}
-
-// acc[0..7] += fma(q_k, scale, bias) for the 8 nibbles of w (packed f32x2 math).
-__device__ __forceinline__ void accumulate_word(uint32_t w, const PairParams &p, float2 (&acc)[4])
-{
-    const uint32_t hi = w >> 12;  // nibbles 5, 6, 7 -> bit positions 8, 12, 16
-    const float2 m23 = make_float2(-kTwo23, -kTwo23);
-    const float2 v01 = __fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23);
-    const float2 v23 = __fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23);
-    const float2 v45 = __fadd2_rn(make_float2(magic_nibble(w, 4), magic_nibble(hi, 2)), m23);
-    const float2 v67 = __fadd2_rn(make_float2(magic_nibble(hi, 3), magic_nibble(hi, 4)), m23);
-    acc[0] = __fadd2_rn(acc[0], __ffma2_rn(v01, p.s01, p.bb));
-    acc[1] = __fadd2_rn(acc[1], __ffma2_rn(v23, p.s23, p.bb));
-    acc[2] = __fadd2_rn(acc[2], __ffma2_rn(v45, p.s42, p.bb));
-    acc[3] = __fadd2_rn(acc[3], __ffma2_rn(v67, p.s34, p.bb));
-}
 
 // Reduce-scatter of E sums over the IS id strides (lane bits 0..log2(IS)-1):
 // afterwards lane `is` holds elements [is * E/IS, (is+1) * E/IS) in acc[0 .. E/IS).
@@ -209,21 +172,42 @@ __device__ __forceinline__ TableView table_view(const BagTables &tabs, int t, in
     return v;
 }
 
-// acc += the E dequantized values of code vector w with packed scale/bias sbw
-template <int E>
-__device__ __forceinline__ void accumulate_row(const typename CodeVec<E>::T &w, uint32_t sbw,
-                                               float2 (&acc2)[E / 2])
+// acc[0..7] = fma(m, fma(q_k, scale, bias), acc) for the 8 nibbles of w: weight m = 1
+// adds the row, m = 0 leaves acc unchanged (x * 0 is a signed zero and acc is never -0).
+// The even nibbles are masked into the low halves of the bytes of lo, the odd ones into
+// hi; a byte permute puts nibble byte b under the exponent byte 0x4B, giving the float
+// 2^23 + q exactly; subtracting 2^23 leaves q, and one fma with the row's scale and bias
+// gives fma(q, scale, bias) bit for bit.
+__device__ __forceinline__ void accumulate_word_w(uint32_t w, float2 ss, float2 bb, float2 m2, float2 (&acc)[4])
 {
-    const PairParams prm = pair_params(sbw);
+    const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+    const float2 m23 = make_float2(-kTwo23, -kTwo23);
 #pragma unroll
-    for (int i = 0; i < E / 8; ++i) {
-        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
-        accumulate_word(CodeVec<E>::word(w, i), prm, quad);
+    for (int b = 0; b < 4; ++b) {
+        const uint32_t sel = 0x7440u | (uint32_t)b;
+        const float2 v = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, sel)),
+                                                __uint_as_float(__byte_perm(hi, 0x4B000000u, sel))), m23);
+        acc[b] = __ffma2_rn(m2, __ffma2_rn(v, ss, bb), acc[b]);
     }
 }
 
-// Sums the ids at positions q, q + step, ... < p1 into acc2 (groups of 4 loads in
-// flight, then single ids). Out-of-range ids are skipped and reported in `bad`.
+template <int E>
+__device__ __forceinline__ void accumulate_row_w(const typename CodeVec<E>::T &w, uint32_t sbw, float m,
+                                                 float2 (&acc2)[E / 2])
+{
+    const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
+    const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
+    const float2 ss = make_float2(S, S), bb = make_float2(B, B), m2 = make_float2(m, m);
+#pragma unroll
+    for (int i = 0; i < E / 8; ++i) {
+        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
+        accumulate_word_w(CodeVec<E>::word(w, i), ss, bb, m2, quad);
+    }
+}
+
+// Sums the ids at positions q, q + step, ... < p1 into acc2, four loads in flight, with
+// no branch per id: an out-of-range id (reported in `bad`) reads row 0 and adds it with
+// weight 0. The table must have a row.
 template <int E>
 __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indices, int32_t q, int32_t p1,
                                                int step, const TableView &tv, float2 (&acc2)[E / 2],
@@ -232,35 +216,33 @@ __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indic
     using V = typename CodeVec<E>::T;
     for (; q + 3 * step < p1; q += 4 * step) {
         uint32_t id[4];
-        bool ok[4];
+        float m[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            id[u] = (uint32_t)__ldg(indices + q + u * step);
-            ok[u] = id[u] < tv.n_rows;
-            bad |= !ok[u];
+            const uint32_t v = (uint32_t)__ldg(indices + q + u * step);
+            const bool ok = v < tv.n_rows;
+            bad |= !ok;
+            m[u] = ok ? 1.0f : 0.0f;
+            id[u] = ok ? v : 0u;
         }
         V w[4];
         uint32_t sbw[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            if (ok[u]) {
-                w[u] = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id[u] * tv.ld));
-                sbw[u] = __ldg(tv.sb + id[u]);
-            }
+            w[u] = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id[u] * tv.ld));
+            sbw[u] = __ldg(tv.sb + id[u]);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            if (ok[u])
-                accumulate_row<E>(w[u], sbw[u], acc2);
+            accumulate_row_w<E>(w[u], sbw[u], m[u], acc2);
     }
     for (; q < p1; q += step) {
-        const uint32_t id = (uint32_t)__ldg(indices + q);
-        if (id < tv.n_rows) {
-            accumulate_row<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)),
-                              __ldg(tv.sb + id), acc2);
-        } else {
-            bad = true;
-        }
+        const uint32_t v = (uint32_t)__ldg(indices + q);
+        const bool ok = v < tv.n_rows;
+        bad |= !ok;
+        const uint32_t id = ok ? v : 0u;
+        accumulate_row_w<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)), __ldg(tv.sb + id),
+                            ok ? 1.0f : 0.0f, acc2);
     }
 }
 
@@ -302,7 +284,10 @@ __device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagA
         for (int k = 0; k < E / 2; ++k)
             acc2[k] = make_float2(0.0f, 0.0f);
         bool bad = false;
-        accumulate_ids<E>(a.indices, p + is, p1, IS, tv, acc2, bad);
+        if (tv.n_rows > 0)
+            accumulate_ids<E>(a.indices, p + is, p1, IS, tv, acc2, bad);
+        else
+            bad = p1 > p;
         if (bad)
             raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
         float acc[E];
@@ -372,34 +357,30 @@ struct ChunkVec<32> {
     }
 };
 
-// The EL dequantized values fma(q, scale, bias) of a chunk, as EL / 4 float4.
+// The EL dequantized values fma(q, scale, bias) of a chunk, as EL / 4 float4 (nibbles
+// to floats by byte permutes, as accumulate_word_w).
 template <int EL>
 __device__ __forceinline__ void dequant_chunk_to(const typename ChunkVec<EL>::T &c, uint32_t sbw, float4 (&x)[EL / 4])
 {
     const float2 m23 = make_float2(-kTwo23, -kTwo23);
     const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
     const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
-    const float2 bb = make_float2(B, B);
-    const float2 s01 = make_float2(S, __fmul_rn(S, 0.0625f));
-    const float2 s23 = make_float2(__fmul_rn(S, 0.00390625f), __fmul_rn(S, 0.000244140625f));
-    if constexpr (EL == 4) {
-        const uint32_t w = ChunkVec<EL>::word(c, 0);
-        const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23), s01, bb);
-        const float2 x23 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23), s23, bb);
-        x[0] = make_float4(x01.x, x01.y, x23.x, x23.y);
-    } else {
-        const float S4 = __fmul_rn(S, 1.52587890625e-05f);
-        const float2 s42 = make_float2(S4, s23.x), s34 = make_float2(s23.y, S4);
+    const float2 ss = make_float2(S, S), bb = make_float2(B, B);
+    constexpr int WORDS = EL >= 8 ? EL / 8 : 1;
+    constexpr int BYTES = EL >= 8 ? 4 : EL / 2;
 #pragma unroll
-        for (int i = 0; i < EL / 8; ++i) {
-            const uint32_t w = ChunkVec<EL>::word(c, i);
-            const uint32_t hi = w >> 12;
-            const float2 x01 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 0), magic_nibble(w, 1)), m23), s01, bb);
-            const float2 x23 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 2), magic_nibble(w, 3)), m23), s23, bb);
-            const float2 x45 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(w, 4), magic_nibble(hi, 2)), m23), s42, bb);
-            const float2 x67 = __ffma2_rn(__fadd2_rn(make_float2(magic_nibble(hi, 3), magic_nibble(hi, 4)), m23), s34, bb);
-            x[2 * i] = make_float4(x01.x, x01.y, x23.x, x23.y);
-            x[2 * i + 1] = make_float4(x45.x, x45.y, x67.x, x67.y);
+    for (int i = 0; i < WORDS; ++i) {
+        const uint32_t w = ChunkVec<EL>::word(c, i);
+        const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+        for (int b = 0; b < BYTES; b += 2) {
+            const uint32_t s0 = 0x7440u | (uint32_t)b, s1 = 0x7440u | (uint32_t)(b + 1);
+            const float2 v0 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, s0)),
+                                                     __uint_as_float(__byte_perm(hi, 0x4B000000u, s0))), m23);
+            const float2 v1 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, s1)),
+                                                     __uint_as_float(__byte_perm(hi, 0x4B000000u, s1))), m23);
+            const float2 x0 = __ffma2_rn(v0, ss, bb), x1 = __ffma2_rn(v1, ss, bb);
+            x[i * 2 + b / 2] = make_float4(x0.x, x0.y, x1.x, x1.y);
         }
     }
 }
