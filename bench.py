@@ -61,10 +61,11 @@ DEVICE_DRAWN = ("production",)   # workloads whose fp32 tables are drawn on the 
 HOST_PARALLEL_BYTES = 256 << 20  # host-drawn workloads above this use a process pool
 HBM_FALLBACK_GBS = 6650.0
 OTHER_WORKLOADS = ("tiny", "kaggle", "terabyte", "sweep-16", "sweep-32", "sweep-64", "sweep-128", "sweep-256")
-# dram bytes read + written per quantized row, from the ncu capture of the quantizer on
-# the largest Kaggle-shaped table (304.1 MB read + 47.4 MB written for 4,742,154 rows);
-# reported only while the kernel source still has the sha256 prefix recorded with it.
-NCU_QUANT_TRAFFIC = {"kernel_sha": "b26922f6dcea3bc2", "bytes_per_row": 74.12}
+# dram bytes read + written per quantized row, by row width d, from ncu captures of the
+# quantizer (d=16: the largest Kaggle-shaped table, 304.1 MB read + 47.4 MB written for
+# 4,742,154 rows). A launch's traffic scales with its rows at a fixed d; it is reported
+# only for a captured d and while the kernel source still has the recorded sha256 prefix.
+NCU_QUANT_TRAFFIC = {"kernel_sha": "b26922f6dcea3bc2", "bytes_per_row": {16: 74.12}}
 
 
 # ---------------------------------------------------------------------------
@@ -519,8 +520,9 @@ def run_gpu(args, wl: W.Workload) -> None:
     q_flops = float(FLOPS_PER_ELEMENT_EVAL * EVALS_PER_ROW * wlr.d) * wlr.total_rows * args.steps
     achieved = q_flops / (tm["quantize"] / 1e3) / 1e12
     traffic = None  # bytes per average quantize launch (one launch per table)
-    if NCU_QUANT_TRAFFIC["kernel_sha"] == _kernel_sha():
-        traffic = NCU_QUANT_TRAFFIC["bytes_per_row"] * wlr.total_rows / max(1, sum(1 for n in wlr.rows if n))
+    per_row = NCU_QUANT_TRAFFIC["bytes_per_row"].get(wlr.d)
+    if per_row is not None and NCU_QUANT_TRAFFIC["kernel_sha"] == _kernel_sha():
+        traffic = per_row * wlr.total_rows / max(1, sum(1 for n in wlr.rows if n))
 
     line = None
     if rank == 0:
