@@ -63,9 +63,10 @@ HBM_FALLBACK_GBS = 6650.0
 OTHER_WORKLOADS = ("tiny", "kaggle", "terabyte", "sweep-16", "sweep-32", "sweep-64", "sweep-128", "sweep-256")
 # dram bytes read + written per quantized row, by row width d, from ncu captures of the
 # quantizer (d=16: the largest Kaggle-shaped table, 304.1 MB read + 47.4 MB written for
-# 4,742,154 rows). A launch's traffic scales with its rows at a fixed d; it is reported
+# 4,742,154 rows; d=128: the sweep d=128 table, 513.4 MB read + 61.7 MB written for
+# 1,000,000 rows). A launch's traffic scales with its rows at a fixed d; it is reported
 # only for a captured d and while the kernel source still has the recorded sha256 prefix.
-NCU_QUANT_TRAFFIC = {"kernel_sha": "b26922f6dcea3bc2", "bytes_per_row": {16: 74.12}}
+NCU_QUANT_TRAFFIC = {"kernel_sha": "b26922f6dcea3bc2", "bytes_per_row": {16: 74.12, 128: 575.09}}
 
 
 # ---------------------------------------------------------------------------

@@ -12,9 +12,12 @@
 // ORs 0x4B000000 onto the nibble left in place at bits 4k..4k+3 (the float
 // 2^23 + q*2^(4k); subtracting 2^23 leaves q*2^(4k) exactly, and an FMA with
 // scale*2^(-4k), an exact power-of-two rescaling, gives fma(q, scale, bias) bit for
-// bit). The lookup masks the even and odd nibbles into the low halves of bytes and
-// byte-permutes each under the exponent byte 0x4B (the float 2^23 + q), which takes
-// one instruction per element and one scale for all of them.
+// bit). The one-hot lookup masks the even and odd nibbles into the low halves of
+// bytes and byte-permutes each under the exponent byte 0x4B (the float 2^23 + q). The
+// long-bag lookup byte-permutes each nibble alone into bits 20..23 of a zero word, the
+// float q * 2^-129 (a subnormal or the least normal binade, exact either way), and
+// multiplies it by scale * 2^129 inside the FMA: one instruction per element before
+// the FMA, and no subtraction.
 #include "dq_internal.cuh"
 
 namespace dq {
@@ -172,13 +175,30 @@ __device__ __forceinline__ TableView table_view(const BagTables &tabs, int t, in
     return v;
 }
 
-// acc[0..7] = fma(m, fma(q_k, scale, bias), acc) for the 8 nibbles of w: weight m = 1
-// adds the row, m = 0 leaves acc unchanged (x * 0 is a signed zero and acc is never -0).
-// The even nibbles are masked into the low halves of the bytes of lo, the odd ones into
-// hi; a byte permute puts nibble byte b under the exponent byte 0x4B, giving the float
-// 2^23 + q exactly; subtracting 2^23 leaves q, and one fma with the row's scale and bias
-// gives fma(q, scale, bias) bit for bit.
-__device__ __forceinline__ void accumulate_word_w(uint32_t w, float2 ss, float2 bb, float2 m2, float2 (&acc)[4])
+// acc[0..7] += fma(q_k, scale, bias) for the 8 nibbles of w, with the nibble placed at
+// bits 20..23 of an otherwise zero word: the float q * 2^-129 exactly (below 2^-126 it
+// is subnormal, the value is the integer word times 2^-149 either way), so
+// fma(q * 2^-129, scale * 2^129, bias) is fma(q, scale, bias) bit for bit (the product
+// is exact). ss = scale * 2^129 must be finite: |scale| < 1/2.
+__device__ __forceinline__ void accumulate_word_d(uint32_t w, float2 ss, float2 bb, float2 (&acc)[4])
+{
+    const uint32_t lo = (w << 4) & 0xF0F0F0F0u, hi = w & 0xF0F0F0F0u;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const uint32_t sel = 0x4044u | ((uint32_t)b << 8);
+        const float2 v = make_float2(__uint_as_float(__byte_perm(lo, 0u, sel)), __uint_as_float(__byte_perm(hi, 0u, sel)));
+        acc[b] = __fadd2_rn(acc[b], __ffma2_rn(v, ss, bb));
+    }
+}
+
+constexpr float kTwo64 = 18446744073709551616.0f, kTwo65 = 36893488147419103232.0f;
+
+// scale * 2^129 for accumulate_word_d: two power-of-two products, exact for |scale| < 1/2.
+__device__ __forceinline__ float scale_up(float S) { return __fmul_rn(__fmul_rn(S, kTwo64), kTwo65); }
+
+// The same sums with the nibble under the exponent byte 0x4B (the float 2^23 + q, minus
+// 2^23): any scale.
+__device__ __forceinline__ void accumulate_word_m(uint32_t w, float2 ss, float2 bb, float2 (&acc)[4])
 {
     const uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
     const float2 m23 = make_float2(-kTwo23, -kTwo23);
@@ -187,27 +207,23 @@ __device__ __forceinline__ void accumulate_word_w(uint32_t w, float2 ss, float2 
         const uint32_t sel = 0x7440u | (uint32_t)b;
         const float2 v = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(lo, 0x4B000000u, sel)),
                                                 __uint_as_float(__byte_perm(hi, 0x4B000000u, sel))), m23);
-        acc[b] = __ffma2_rn(m2, __ffma2_rn(v, ss, bb), acc[b]);
+        acc[b] = __fadd2_rn(acc[b], __ffma2_rn(v, ss, bb));
     }
 }
 
-template <int E>
-__device__ __forceinline__ void accumulate_row_w(const typename CodeVec<E>::T &w, uint32_t sbw, float m,
-                                                 float2 (&acc2)[E / 2])
+// Scale and bias of a row as floats; an id outside the table (ok false) gets 0 and 0,
+// so its row adds +0 (the sums never hold -0).
+__device__ __forceinline__ void row_sb(uint32_t sbw, bool ok, float &S, float &B)
 {
-    const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
-    const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
-    const float2 ss = make_float2(S, S), bb = make_float2(B, B), m2 = make_float2(m, m);
-#pragma unroll
-    for (int i = 0; i < E / 8; ++i) {
-        float2 (&quad)[4] = *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]);
-        accumulate_word_w(CodeVec<E>::word(w, i), ss, bb, m2, quad);
-    }
+    sbw = ok ? sbw : 0u;
+    S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
+    B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
 }
 
 // Sums the ids at positions q, q + step, ... < p1 into acc2, four loads in flight, with
-// no branch per id: an out-of-range id (reported in `bad`) reads row 0 and adds it with
-// weight 0. The table must have a row.
+// no branch per id: an out-of-range id (reported in `bad`) reads row 0 and adds +0.
+// The table must have a row. A group whose rows all have |scale| < 1/2 takes the
+// scaled-subnormal decode, any other the exponent-byte decode.
 template <int E>
 __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indices, int32_t q, int32_t p1,
                                                int step, const TableView &tv, float2 (&acc2)[E / 2],
@@ -216,14 +232,13 @@ __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indic
     using V = typename CodeVec<E>::T;
     for (; q + 3 * step < p1; q += 4 * step) {
         uint32_t id[4];
-        float m[4];
+        bool ok[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const uint32_t v = (uint32_t)__ldg(indices + q + u * step);
-            const bool ok = v < tv.n_rows;
-            bad |= !ok;
-            m[u] = ok ? 1.0f : 0.0f;
-            id[u] = ok ? v : 0u;
+            ok[u] = v < tv.n_rows;
+            bad |= !ok[u];
+            id[u] = ok[u] ? v : 0u;
         }
         V w[4];
         uint32_t sbw[4];
@@ -232,17 +247,44 @@ __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indic
             w[u] = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id[u] * tv.ld));
             sbw[u] = __ldg(tv.sb + id[u]);
         }
+        float S[4], B[4];
+        bool small = true;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-            accumulate_row_w<E>(w[u], sbw[u], m[u], acc2);
+        for (int u = 0; u < 4; ++u) {
+            row_sb(sbw[u], ok[u], S[u], B[u]);
+            small &= fabsf(S[u]) < 0.5f;
+        }
+        if (small) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float Sp = scale_up(S[u]);
+                const float2 ss = make_float2(Sp, Sp), bb = make_float2(B[u], B[u]);
+#pragma unroll
+                for (int i = 0; i < E / 8; ++i)
+                    accumulate_word_d(CodeVec<E>::word(w[u], i), ss, bb, *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]));
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float2 ss = make_float2(S[u], S[u]), bb = make_float2(B[u], B[u]);
+#pragma unroll
+                for (int i = 0; i < E / 8; ++i)
+                    accumulate_word_m(CodeVec<E>::word(w[u], i), ss, bb, *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]));
+            }
+        }
     }
     for (; q < p1; q += step) {
         const uint32_t v = (uint32_t)__ldg(indices + q);
         const bool ok = v < tv.n_rows;
         bad |= !ok;
         const uint32_t id = ok ? v : 0u;
-        accumulate_row_w<E>(__ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld)), __ldg(tv.sb + id),
-                            ok ? 1.0f : 0.0f, acc2);
+        const V w = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id * tv.ld));
+        float S, B;
+        row_sb(__ldg(tv.sb + id), ok, S, B);
+        const float2 ss = make_float2(S, S), bb = make_float2(B, B);
+#pragma unroll
+        for (int i = 0; i < E / 8; ++i)
+            accumulate_word_m(CodeVec<E>::word(w, i), ss, bb, *reinterpret_cast<float2(*)[4]>(&acc2[4 * i]));
     }
 }
 
@@ -358,7 +400,7 @@ struct ChunkVec<32> {
 };
 
 // The EL dequantized values fma(q, scale, bias) of a chunk, as EL / 4 float4 (nibbles
-// to floats by byte permutes, as accumulate_word_w).
+// to floats by byte permutes under the exponent byte, as accumulate_word_m).
 template <int EL>
 __device__ __forceinline__ void dequant_chunk_to(const typename ChunkVec<EL>::T &c, uint32_t sbw, float4 (&x)[EL / 4])
 {

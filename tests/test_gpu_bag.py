@@ -70,6 +70,35 @@ def test_bag_matches_oracle(cuda_device, d, pool):
         assert np.array_equal(got.view(np.uint32), ref.view(np.uint32))
 
 
+def _scaled_table(n, d, seed, scales):
+    """A random packed table whose rows cycle through the given binary16 scales."""
+    codes, sb = _packed(n, d, seed, ((d + 1) // 2 + 15) // 16 * 16)
+    s = np.asarray(scales, np.float16)[np.arange(n) % len(scales)]
+    sb[:, 0] = s.view(np.uint16)
+    return codes, sb
+
+
+@pytest.mark.parametrize("d", [16, 64, 128, 256])
+def test_bag_rows_of_every_scale(cuda_device, d):
+    """Bags averaging 6 ids (the long-bag layout), some of one id, over rows whose
+    binary16 scales run from zero and subnormals through 1/2 to 60000, both signs: a
+    group of rows takes the scaled-subnormal decode only while every |scale| < 1/2, the
+    exponent-byte decode otherwise, and both must sum fma(q, scale, bias)."""
+    scales = [0.0, -0.0, 6e-8, 1e-4, 0.01, 0.4998, 0.5, 0.5005, 1.0, 3.0, 250.0, 60000.0, -0.3, -0.7, -2.0]
+    T, B = 2, 64
+    rows = [300, 77]
+    tabs = [_scaled_table(n, d, 40 + t, scales) for t, n in enumerate(rows)]
+    for seed, (lo, hi) in ((d, (0, 12)), (d + 1, (4, 8))):
+        idx, off = _bags(T, B, rows, lo, hi, seed)
+        got, _ = _gpu_bag(tabs, d, idx, off, B)
+        ref, mag, skipped = oracle.embbag(tabs, d, idx, off, B, with_abs_sum=True)
+        assert skipped == 0
+        bag_tolerance_check(got, ref, mag)
+        lens = np.diff(off.astype(np.int64)).reshape(T, B).T          # [B, T]
+        one = np.repeat(lens == 1, d, axis=1)
+        assert np.array_equal(got[one].view(np.uint32), ref[one].view(np.uint32))
+
+
 def test_bag_bad_ids_and_offsets(cuda_device):
     d, T, B = 64, 2, 50
     rows = [100, 100]
