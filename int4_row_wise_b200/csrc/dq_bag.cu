@@ -9,21 +9,29 @@
 // Both kernels are bound by HBM (and, for long bags, by instruction issue): packed
 // rows are read with 8- or 16-byte vector loads, outputs written with 16-byte stores.
 // A nibble becomes a float without integer-to-float conversion. The dequantize kernel
-// ORs 0x4B000000 onto the nibble left in place at bits 4k..4k+3 (the float
+// and the long-bag lookup byte-permute each nibble alone into bits 20..23 of a zero
+// word, the float q * 2^-129 (a subnormal or the least normal binade, exact either
+// way), and multiply it by scale * 2^129 inside the FMA: one instruction per element
+// before the FMA, and no subtraction; rows with |scale| >= 1/2, where scale * 2^129
+// would overflow, take an exponent trick instead. The dequantize kernel's fallback ORs
+// 0x4B000000 onto the nibble left in place at bits 4k..4k+3 (the float
 // 2^23 + q*2^(4k); subtracting 2^23 leaves q*2^(4k) exactly, and an FMA with
 // scale*2^(-4k), an exact power-of-two rescaling, gives fma(q, scale, bias) bit for
-// bit). The one-hot lookup masks the even and odd nibbles into the low halves of
-// bytes and byte-permutes each under the exponent byte 0x4B (the float 2^23 + q). The
-// long-bag lookup byte-permutes each nibble alone into bits 20..23 of a zero word, the
-// float q * 2^-129 (a subnormal or the least normal binade, exact either way), and
-// multiplies it by scale * 2^129 inside the FMA: one instruction per element before
-// the FMA, and no subtraction.
+// bit). The one-hot lookup and the long-bag fallback mask the even and odd nibbles
+// into the low halves of bytes and byte-permute each under the exponent byte 0x4B
+// (the float 2^23 + q).
 #include "dq_internal.cuh"
 
 namespace dq {
 namespace {
 
 constexpr float kTwo23 = 8388608.0f;
+constexpr float kTwo64 = 18446744073709551616.0f, kTwo65 = 36893488147419103232.0f;
+
+// scale * 2^129, the factor that turns the subnormal q * 2^-129 (a nibble placed at bits
+// 20..23 of a zero word) back into q * scale inside an FMA: two power-of-two products,
+// exact for |scale| < 1/2.
+__device__ __forceinline__ float scale_up(float S) { return __fmul_rn(__fmul_rn(S, kTwo64), kTwo65); }
 
 struct RowParams {
     float s[5];   // scale * 2^(-4k), k = 0..4
@@ -61,27 +69,37 @@ __device__ __forceinline__ void decode_word(uint32_t w, const RowParams &p, floa
 }
 
 // ---------------------------------------------------------------------------
-// dequantize: one thread per 16-element chunk (8 code bytes -> 64 output bytes)
+// dequantize: one thread per 4 elements (2 code bytes -> one 16-byte store), so that a
+// warp's store covers 512 contiguous bytes
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) dequant16_kernel(const DequantArgs a)
+__global__ void __launch_bounds__(256) dequant16_kernel(const DequantArgs a, const int cpr_log2)
 {
-    const int cpr = a.d / 16;
-    const int64_t total = a.n * cpr;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total;
-         c += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t row = c / cpr;
+    // one float4 of output per thread: a warp's store covers 512 contiguous bytes
+    const int cpr = a.d / 4;
+    const uint64_t total = (uint64_t)a.n * cpr;
+    for (uint64_t c = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; c < total;
+         c += (uint64_t)gridDim.x * blockDim.x) {
+        const uint64_t row = cpr_log2 >= 0 ? c >> cpr_log2 : c / (uint64_t)cpr;
         const int part = (int)(c - row * cpr);
-        const uint2 w = __ldg(reinterpret_cast<const uint2 *>(a.codes + row * a.codes_ld) + part);
+        const uint32_t w = __ldg(reinterpret_cast<const uint16_t *>(a.codes + row * a.codes_ld) + part);
         const uint32_t sbw = __ldg(reinterpret_cast<const uint32_t *>(a.scale_bias) + row);
-        const RowParams p = row_params(sbw);
-        float x0[8], x1[8];
-        decode_word(w.x, p, x0);
-        decode_word(w.y, p, x1);
-        float4 *o = reinterpret_cast<float4 *>(a.out + row * a.out_ld) + part * 4;
-        __stcs(o + 0, make_float4(x0[0], x0[1], x0[2], x0[3]));
-        __stcs(o + 1, make_float4(x0[4], x0[5], x0[6], x0[7]));
-        __stcs(o + 2, make_float4(x1[0], x1[1], x1[2], x1[3]));
-        __stcs(o + 3, make_float4(x1[4], x1[5], x1[6], x1[7]));
+        const float S = __half2float(__ushort_as_half((unsigned short)(sbw & 0xffffu)));
+        const float B = __half2float(__ushort_as_half((unsigned short)(sbw >> 16)));
+        float4 x;
+        if (fabsf(S) < 0.5f) {
+            const float Sp = scale_up(S);
+            const uint32_t lo = (w << 4) & 0xF0F0u, hi = w & 0xF0F0u;
+            x.x = __fmaf_rn(__uint_as_float(__byte_perm(lo, 0u, 0x4044u)), Sp, B);
+            x.y = __fmaf_rn(__uint_as_float(__byte_perm(hi, 0u, 0x4044u)), Sp, B);
+            x.z = __fmaf_rn(__uint_as_float(__byte_perm(lo, 0u, 0x4144u)), Sp, B);
+            x.w = __fmaf_rn(__uint_as_float(__byte_perm(hi, 0u, 0x4144u)), Sp, B);
+        } else {
+            const RowParams p = row_params(sbw);
+            float x0[8];
+            decode_word(w, p, x0);
+            x = make_float4(x0[0], x0[1], x0[2], x0[3]);
+        }
+        __stcs(reinterpret_cast<float4 *>(a.out + row * a.out_ld) + part, x);
     }
 }
 
@@ -109,9 +127,10 @@ __global__ void __launch_bounds__(256) dequant_generic_kernel(const DequantArgs 
 //
 // Two layouts in one kernel, chosen on the device from the id count (the last
 // offset), so the host need not know the pooling:
-//  - long bags (average pooling >= 4): one warp per bag; its ids are read 32 at a
-//    time (the first 32 one bag ahead), repeated ids merged, distinct rows spread
-//    over the warp's slots, partial sums added through shared memory;
+//  - long bags (average pooling >= 4): d / E lanes cover a row (E elements, E / 2
+//    code bytes each) and IS such lane groups take every IS-th id of the same bag,
+//    four ids in flight and the next four ids loaded ahead; the IS partial sums meet
+//    in a reduce-scatter over shuffles, and each lane stores E / IS finished sums;
 //  - short bags (one-hot lookups): a warp takes 32 bags, each lane writes 16-byte
 //    chunks of whole output rows straight from registers.
 // Either way a bag's sum is binary32 accumulation of the binary32 fma(q, s, b)
@@ -191,11 +210,6 @@ __device__ __forceinline__ void accumulate_word_d(uint32_t w, float2 ss, float2 
     }
 }
 
-constexpr float kTwo64 = 18446744073709551616.0f, kTwo65 = 36893488147419103232.0f;
-
-// scale * 2^129 for accumulate_word_d: two power-of-two products, exact for |scale| < 1/2.
-__device__ __forceinline__ float scale_up(float S) { return __fmul_rn(__fmul_rn(S, kTwo64), kTwo65); }
-
 // The same sums with the nibble under the exponent byte 0x4B (the float 2^23 + q, minus
 // 2^23): any scale.
 __device__ __forceinline__ void accumulate_word_m(uint32_t w, float2 ss, float2 bb, float2 (&acc)[4])
@@ -230,15 +244,21 @@ __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indic
                                                bool &bad)
 {
     using V = typename CodeVec<E>::T;
+    // the ids of the next group of four are loaded while the current group is summed
+    uint32_t nxt[4];
+    if (q + 3 * step < p1) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            nxt[u] = (uint32_t)__ldg(indices + q + u * step);
+    }
     for (; q + 3 * step < p1; q += 4 * step) {
         uint32_t id[4];
         bool ok[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-            const uint32_t v = (uint32_t)__ldg(indices + q + u * step);
-            ok[u] = v < tv.n_rows;
+            ok[u] = nxt[u] < tv.n_rows;
             bad |= !ok[u];
-            id[u] = ok[u] ? v : 0u;
+            id[u] = ok[u] ? nxt[u] : 0u;
         }
         V w[4];
         uint32_t sbw[4];
@@ -246,6 +266,11 @@ __device__ __forceinline__ void accumulate_ids(const int32_t *__restrict__ indic
         for (int u = 0; u < 4; ++u) {
             w[u] = __ldg(reinterpret_cast<const V *>(tv.codes + (uint64_t)id[u] * tv.ld));
             sbw[u] = __ldg(tv.sb + id[u]);
+        }
+        if (q + 7 * step < p1) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                nxt[u] = (uint32_t)__ldg(indices + q + (4 + u) * step);
         }
         float S[4], B[4];
         bool small = true;
@@ -659,12 +684,16 @@ int grid_for(int64_t work, int block, int num_sms)
 
 cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t stream)
 {
-    const bool fast = a.d % 16 == 0 && a.codes_ld % 8 == 0 && a.out_ld % 4 == 0 &&
-                      (reinterpret_cast<uintptr_t>(a.codes) & 7) == 0 &&
+    const bool fast = a.d % 4 == 0 && a.codes_ld % 2 == 0 && a.out_ld % 4 == 0 &&
+                      (reinterpret_cast<uintptr_t>(a.codes) & 1) == 0 &&
                       (reinterpret_cast<uintptr_t>(a.out) & 15) == 0 &&
                       (reinterpret_cast<uintptr_t>(a.scale_bias) & 3) == 0;
     if (fast)
-        dequant16_kernel<<<grid_for(a.n * (a.d / 16), 256, num_sms), 256, 0, stream>>>(a);
+    {
+        const int cpr = a.d / 4;   // float4 chunks per row; a power of two is a shift
+        const int lg = (cpr & (cpr - 1)) == 0 ? 31 - __builtin_clz((unsigned)cpr) : -1;
+        dequant16_kernel<<<grid_for(a.n * cpr, 256, num_sms), 256, 0, stream>>>(a, lg);
+    }
     else
         dequant_generic_kernel<<<grid_for(a.n * ((a.d + 1) / 2), 256, num_sms), 256, 0, stream>>>(a);
     return cudaGetLastError();

@@ -20,7 +20,8 @@ def _packed(n, d, seed, codes_ld=None):
 
 
 @pytest.mark.parametrize("d,codes_ld,out_ld", [(16, 8, 16), (128, 64, 128), (256, 128, 256), (32, 16, 32),
-                                               (7, 4, 7), (16, 9, 16), (64, 32, 65), (1, 1, 1), (48, 24, 48)])
+                                               (7, 4, 7), (16, 9, 16), (64, 32, 65), (1, 1, 1), (48, 24, 48),
+                                               (100, 50, 100), (12, 6, 12), (20, 10, 24)])
 def test_dequantize_bit_exact(cuda_device, d, codes_ld, out_ld):
     n = 5003
     codes, sb = _packed(n, d, d, codes_ld)
@@ -76,6 +77,20 @@ def _scaled_table(n, d, seed, scales):
     s = np.asarray(scales, np.float16)[np.arange(n) % len(scales)]
     sb[:, 0] = s.view(np.uint16)
     return codes, sb
+
+
+@pytest.mark.parametrize("d", [16, 48, 128])
+def test_dequantize_rows_of_every_scale(cuda_device, d):
+    """Rows whose binary16 scales run from zero and subnormals through 1/2 to 60000, both
+    signs: rows with |scale| < 1/2 take the scaled-subnormal decode, the others the
+    exponent-byte decode; both must give fma(q, scale, bias) bit for bit."""
+    scales = [0.0, -0.0, 6e-8, 1e-4, 0.01, 0.4998, 0.5, 0.5005, 1.0, 3.0, 250.0, 60000.0, -0.3, -0.7, -2.0]
+    n = 3001
+    codes, sb = _scaled_table(n, d, 77, scales)
+    want = oracle.dequantize_rows(codes, sb, d)
+    out = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    dq.dq_dequantize_rows(to_dev(codes), codes.shape[1], to_dev(sb.view(np.int16)), n, d, out, d)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
 
 
 @pytest.mark.parametrize("d", [16, 64, 128, 256])
