@@ -564,8 +564,10 @@ def run_gpu(args, wl: W.Workload) -> None:
                      for c, s in zip(step.codes, step.sbs)]
         line["cpu_baseline"] = OracleBench(wlr, host_tabs).baseline(args.ref_seconds)
         del host_tabs
-    if rank == 0 and not args.no_e2e:
-        line["e2e"] = run_e2e(args, wlr, xs, step, dev, dq, world)
+    if not args.no_e2e:   # every rank: the same end-to-end step at N GPUs, max over ranks
+        e2e = run_e2e(args, wlr, xs, step, dev, dq, world)
+        if rank == 0:
+            line["e2e"] = e2e
     del step, xs
     torch.cuda.empty_cache()
     if rank == 0 and world == 1 and not args.no_per_workload:
@@ -755,9 +757,15 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
     ring_chunk = 64 << 20
     need = in_bytes + code_bytes + 4 * ring_chunk + (1 << 30)
     avail = psutil.virtual_memory().available
-    if need * world > 0.8 * avail:
+    fits = need * world <= 0.8 * avail
+    if world > 1:   # one decision for all ranks, so that they take the same collectives
+        import torch.distributed as dist
+        f = torch.tensor([1 if fits else 0], dtype=torch.int32, device=dev)
+        dist.all_reduce(f, op=dist.ReduceOp.MIN)
+        fits = bool(f.item())
+    if not fits:
         return {"skipped": f"pinned host copies of {need / 1e9:.1f} GB per rank x {world} ranks exceed 80 % of the "
-                           f"{avail / 1e9:.0f} GB of free host memory"}
+                           f"free host memory ({avail / 1e9:.0f} GB on rank's node)"}
     stream = step.stream
     host_x = [torch.empty(x.shape, dtype=torch.float32, pin_memory=True) for x in xs]
     for h, x in zip(host_x, xs):
@@ -830,6 +838,10 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
     for k in range(2):
         one(k)
     torch.cuda.synchronize(dev)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for k in range(steps):
