@@ -7,9 +7,9 @@
 // xhat = fma(q, scale, bias) and both sums in binary64.
 //
 // HBM-bound: a row is read once (4d bytes of x, (d+1)/2 code bytes, 4 bytes of
-// scale/bias) by G lanes, each taking 4 consecutive elements per step (a 16-byte
-// load of x and 2 code bytes); a warp keeps 4 row blocks' loads in flight, and
-// binary64 partial sums meet in an XOR butterfly.
+// scale/bias) by G lanes (1 to 8, fewer than the row's 4-element chunks), each taking 4
+// consecutive elements per step (a 16-byte load of x and 2 code bytes); a warp keeps 4
+// row blocks' loads in flight, and binary64 partial sums meet in an XOR butterfly.
 #include "dq_internal.cuh"
 
 namespace dq {
@@ -143,18 +143,19 @@ cudaError_t launch_g(const L2Args &a, int num_sms, cudaStream_t stream)
 
 cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream)
 {
+    // lanes per row: few, so that a lane takes several 4-element chunks of a row and the
+    // per-row work (the binary64 butterfly over the row's lanes, the division and square
+    // root) is shared by more rows per warp; two lanes read a full 32-byte sector of x
+    // per step (measured on the B200: d = 16 best with one lane per row, d = 64 and 128
+    // with two, d = 256 with two or four)
     const int chunks = (a.d + 3) / 4;  // 4 elements per lane and step
-    if (chunks <= 1)
-        return launch_g<1>(a, num_sms, stream);
-    if (chunks <= 2)
-        return launch_g<2>(a, num_sms, stream);
     if (chunks <= 4)
+        return launch_g<1>(a, num_sms, stream);
+    if (chunks <= 32)
+        return launch_g<2>(a, num_sms, stream);
+    if (chunks <= 128)
         return launch_g<4>(a, num_sms, stream);
-    if (chunks <= 8)
-        return launch_g<8>(a, num_sms, stream);
-    if (chunks <= 16)
-        return launch_g<16>(a, num_sms, stream);
-    return launch_g<32>(a, num_sms, stream);
+    return launch_g<8>(a, num_sms, stream);
 }
 
 } // namespace dq
