@@ -62,11 +62,13 @@ HOST_PARALLEL_BYTES = 256 << 20  # host-drawn workloads above this use a process
 HBM_FALLBACK_GBS = 6650.0
 OTHER_WORKLOADS = ("tiny", "kaggle", "terabyte", "sweep-16", "sweep-32", "sweep-64", "sweep-128", "sweep-256")
 # dram bytes read + written per quantized row, by row width d, from ncu captures of the
-# quantizer (d=16: the largest Kaggle-shaped table, 304.1 MB read + 47.4 MB written for
-# 4,742,154 rows; d=128: the sweep d=128 table, 513.4 MB read + 61.7 MB written for
-# 1,000,000 rows). A launch's traffic scales with its rows at a fixed d; it is reported
-# only for a captured d and while the kernel source still has the recorded sha256 prefix.
-NCU_QUANT_TRAFFIC = {"kernel_sha": "b26922f6dcea3bc2", "bytes_per_row": {16: 74.12, 128: 575.09}}
+# quantizer (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:quantize_rows
+# -s 3 -c 1` around `bench.py --workload W --steps 1 --warmup 3 --no-per-workload --no-e2e
+# --no-cpu-baseline --no-next-rows`): d=16, a Kaggle-shaped table of 3,097,041 rows, 199.1 MB
+# read + 25.9 MB written; d=128, the sweep d=128 table of 1,000,000 rows, 514.8 MB read +
+# 61.5 MB written. A launch's traffic scales with its rows at a fixed d; it is reported only
+# for a captured d and while the kernel source still has the recorded sha256 prefix.
+NCU_QUANT_TRAFFIC = {"kernel_sha": "76c38611eb740cec", "bytes_per_row": {16: 72.65, 128: 576.29}}
 
 
 # ---------------------------------------------------------------------------

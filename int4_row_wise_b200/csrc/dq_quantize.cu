@@ -585,9 +585,12 @@ cudaError_t launch_requant_mw(const RequantArgs &a, int64_t max_rows, int greedy
                               cudaStream_t stream)
 {
     constexpr int kBlock = 128;
-    // grid-stride over at most max_rows rows: enough blocks to fill every SM a few times
+    // one lane group per row of the host's bound (max_rows): the blocks past the listed
+    // rows exit at once, and the hardware balances the rest as for the plain quantizer
+    // (a capped grid-stride loop left a ragged last round per warp); the grid-stride
+    // loop stays for bounds above the grid limit
     const int64_t need = (max_rows * W + kBlock - 1) / kBlock;
-    const int64_t cap = (int64_t)num_sms * 16;
+    const int64_t cap = (int64_t)num_sms * 4096;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     const bool full = a.d == M * W;
     bool vec = full && (M % 4 == 0) && (a.grad_ld % 4 == 0) &&
