@@ -748,8 +748,8 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
     (one cudaMemcpyAsync per table), quantizes and dequantizes it, and downloads its
     codes, scale/bias and dequantized rows (those through a ring of pinned chunks, one
     cudaMemcpyAsync per chunk), then makes the lookup call and downloads its output.
-    Uploads, kernels and downloads run on three streams, so table t's upload overlaps
-    table t-1's kernels and table t-2's downloads."""
+    Uploads, kernels and downloads run on three streams over pieces of at most 1M rows, so
+    piece p's upload overlaps piece p-1's kernels and piece p-2's downloads."""
     import psutil
     import torch
     d, T = wl.d, wl.n_tables
@@ -782,8 +782,11 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
     bi_d = torch.empty(max(i.numel() for i, _ in pin_b), dtype=torch.int32, device=dev)
     bo_d = torch.empty(pin_b[0][1].numel(), dtype=torch.int32, device=dev)
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
-    order = sorted(range(T), key=lambda t: wl.rows[t])  # small tables first: short pipeline fill
-    done = [torch.cuda.Event() for _ in range(T)]
+    # pieces of at most 1M rows: piece p's upload overlaps piece p-1's kernels and piece p-2's
+    # downloads, so the pipeline fills and drains in one piece rather than one table
+    piece_rows = 1 << 20
+    pieces = [(t, r0, min(r0 + piece_rows, wl.rows[t])) for t in range(T) for r0 in range(0, wl.rows[t], piece_rows)]
+    done = [torch.cuda.Event() for _ in pieces]
     for e in done:
         e.record(stream)
     tables = [dq.PackedTable(c, s_) for c, s_ in zip(step.codes, step.sbs)]
@@ -802,23 +805,24 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
             bi_d[:n_ids].copy_(bi, non_blocking=True)
             bo_d.copy_(bo, non_blocking=True)
         slot = 0
-        for t in order:
-            n = wl.rows[t]
-            s_in.wait_event(done[t])   # the previous step's kernels of table t have read its input
+        for pi, (t, r0, r1) in enumerate(pieces):
+            n = r1 - r0
+            s_in.wait_event(done[pi])   # the previous step's kernels of this piece have read its input
             with torch.cuda.stream(s_in):
-                xs[t].copy_(host_x[t], non_blocking=True)
+                xs[t][r0:r1].copy_(host_x[t][r0:r1], non_blocking=True)
                 up = torch.cuda.Event()
                 up.record(s_in)
             stream.wait_event(up)
-            dq.dq_quantize_rows_int4(xs[t], n, d, d, step.codes[t], cld, step.sbs[t], None, None,
+            codes_p, sbs_p, deq_p = step.codes[t][r0:r1], step.sbs[t][r0:r1], deq[t][r0:r1]
+            dq.dq_quantize_rows_int4(xs[t][r0:r1], n, d, d, codes_p, cld, sbs_p, None, None,
                                      dq.DQ_MODE_GREEDY, None, stream)
-            dq.dq_dequantize_rows(step.codes[t], cld, step.sbs[t], n, d, deq[t], d, stream)
-            done[t].record(stream)
-            s_out.wait_event(done[t])
+            dq.dq_dequantize_rows(codes_p, cld, sbs_p, n, d, deq_p, d, stream)
+            done[pi].record(stream)
+            s_out.wait_event(done[pi])
             with torch.cuda.stream(s_out):
-                h_codes[t].copy_(step.codes[t], non_blocking=True)
-                h_sb[t].copy_(step.sbs[t], non_blocking=True)
-                flat = deq[t].view(-1)
+                h_codes[t][r0:r1].copy_(codes_p, non_blocking=True)
+                h_sb[t][r0:r1].copy_(sbs_p, non_blocking=True)
+                flat = deq_p.reshape(-1)
                 for c0 in range(0, flat.numel(), per_chunk):
                     c1 = min(flat.numel(), c0 + per_chunk)
                     ring[slot % len(ring)][:c1 - c0].copy_(flat[c0:c1], non_blocking=True)
@@ -855,8 +859,9 @@ def run_e2e(args, wl, xs, step, dev, dq, world) -> dict:
     torch.cuda.empty_cache()
     return {"value": wl.total_rows * world / (ms / 1e3), "unit": "rows/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": ms, "steps": steps,
-            "api": "int4_row_wise_b200.dq_* from pinned host buffers; one cudaMemcpyAsync per table upload and per "
-                   "64 MB chunk of dequantized rows; upload / kernels / download on 3 streams"}
+            "api": "int4_row_wise_b200.dq_* from pinned host buffers, in pieces of at most 1M rows; one "
+                   "cudaMemcpyAsync per piece upload and per 64 MB chunk of dequantized rows; upload / kernels / "
+                   "download on 3 streams"}
 
 
 # ---------------------------------------------------------------------------
