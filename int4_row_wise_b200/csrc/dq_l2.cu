@@ -8,8 +8,9 @@
 //
 // HBM-bound: a row is read once (4d bytes of x, (d+1)/2 code bytes, 4 bytes of
 // scale/bias) by G lanes (1 to 8, fewer than the row's 4-element chunks), each taking 4
-// consecutive elements per step (a 16-byte load of x and 2 code bytes); a warp keeps 4
-// row blocks' loads in flight, and binary64 partial sums meet in an XOR butterfly.
+// consecutive elements per step (a 16-byte load of x and 2 code bytes); a lane works on
+// one row at a time (measured faster than 2, 4 or 8 rows in flight per lane: fewer
+// registers, more resident warps), and binary64 partial sums meet in an XOR butterfly.
 #include "dq_internal.cuh"
 
 namespace dq {
@@ -127,7 +128,7 @@ cudaError_t launch_g(const L2Args &a, int num_sms, cudaStream_t stream)
 {
     const bool vec = a.d % 4 == 0 && a.ld % 4 == 0 && (reinterpret_cast<uintptr_t>(a.x) & 15) == 0 &&
                      a.codes_ld % 2 == 0 && (reinterpret_cast<uintptr_t>(a.codes) & 1) == 0;
-    constexpr int kU = 4;
+    constexpr int kU = 1;
     const int64_t rows_per_block = 256 / G * kU;
     const int64_t need = (a.n + rows_per_block - 1) / rows_per_block;
     const int64_t cap = (int64_t)num_sms * 8;
