@@ -1146,6 +1146,40 @@ def run_sharded(args, wl: W.Workload) -> None:
         torch.cuda.synchronize(dev)
         dist.barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
+
+    # the lookup and the exchange alone, from each owner's global batch of its tables:
+    # through NCCL (sharded_embbag: lookup, all-to-all, reassembly) and folded into the
+    # lookup (sharded_embbag_direct: one kernel stores every row in its owner's buffer)
+    from int4_row_wise_b200.sharded import OwnerBuffers, sharded_embbag, sharded_embbag_direct
+    gwl = W.dataclasses.replace(W.workload(wl.name, seed=100 + rank), batch=world * B)
+    gidx, goff = W.lookup_batch(gwl, batch_id=0)
+    GB = world * B
+    parts, lens = [], []
+    for t in mine:
+        o = goff[t * GB:(t + 1) * GB + 1].astype(np.int64)
+        parts.append(gidx[o[0]:o[-1]])
+        lens.append(np.diff(o))
+    g_idx = torch.from_numpy(np.concatenate(parts) if parts else np.zeros(1, np.int32)).to(dev)
+    g_off = torch.from_numpy(np.concatenate([[0], np.cumsum(np.concatenate(lens))]).astype(np.int32)
+                             if lens else np.zeros(1, np.int32)).to(dev)
+    bufs = OwnerBuffers.create(B, wl.n_tables * d, dev)
+    legs = {}
+    for name, fn in (("nccl", lambda: sharded_embbag(tables, owner, d, g_idx, g_off, GB)),
+                     ("direct", lambda: sharded_embbag_direct(tables, owner, d, g_idx, g_off, GB, bufs))):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        f1.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        legs[name] = max_over_ranks(f0.elapsed_time(f1) / args.steps, dev)
+    del bufs
     ids_local = float(np.mean([n for _, n in batches]))
     bytes_ids = ids_local * 4 + wl.n_tables * B * 4          # ids + bag lengths each rank sends per call
     bytes_out = B * wl.n_tables * d * 4                        # pooled rows each rank receives per call
@@ -1165,6 +1199,13 @@ def run_sharded(args, wl: W.Workload) -> None:
                          "cross_rank_bytes_per_rank_per_call": int((bytes_ids + bytes_out) * cross),
                          "parts": {"ids_and_lengths": int(bytes_ids), "pooled_rows": int(bytes_out)},
                          "note": "at one rank every exchange is a local copy"},
+            "lookup_and_exchange": {
+                "what": "from each owner's global batch of its tables: the lookup and the delivery of every "
+                        "pooled row to its owner's [batch, T*d] rows",
+                "nccl_ms": legs["nccl"], "direct_ms": legs["direct"],
+                "nccl": "dq_embbag_int4_fwd, all_to_all_single, reassembly in table order",
+                "direct": "dq_embbag_int4_fwd_to_owners storing into every owner's buffer (CUDA IPC across ranks), "
+                          "a barrier before and after"},
             "clocks": clocks.summary()}), flush=True)
     dist.barrier()
     dist.destroy_process_group()

@@ -74,6 +74,7 @@ enum {
 
 #define DQ_MAX_D 1024
 #define DQ_MAX_TABLES 64
+#define DQ_MAX_DEST 64
 
 /* One packed table for the embedding bag. codes and scale_bias are device
  * pointers in the packed row format above. */
@@ -151,6 +152,35 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
 dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d,
                              const int32_t *indices, const int32_t *offsets, int32_t batch,
                              float *out, uint32_t *d_flags, void *cuda_stream);
+
+/*
+ * dq_embbag_int4_fwd_to_owners -- the same lookup, each pooled row stored straight into
+ * the buffer of the rank that owns its sample, at its place among all ranks' tables:
+ * the lookup and the exchange of table-wise sharding in one kernel ("Deep Learning
+ * Recommendation Model for Personalization and Recommendation Systems", 提出的方法 /
+ * proposed method: embedding tables model-parallel, the pooled embeddings sent to the
+ * data-parallel ranks; there the exchange is an all-to-all, here each rank writes its
+ * rows into the owners' memory).
+ *
+ *   tables ... batch, d_flags   as dq_embbag_int4_fwd (batch: the global batch)
+ *   table_slot  HOST int32 [n_tables]: the column block of each local table among the
+ *               t_out tables of the output rows; distinct, in [0, t_out)
+ *   t_out       tables in an output row (all ranks' tables), n_tables..DQ_MAX_TABLES*DQ_MAX_DEST
+ *   dest        HOST array of n_dest device pointers (1..DQ_MAX_DEST, copied at the call):
+ *               dest[r] is rank r's buffer [batch / n_dest][t_out*d] binary32, which may be
+ *               another GPU's memory mapped into this process (peer access enabled)
+ *   n_dest      ranks; batch must be a multiple of n_dest
+ *
+ * Bag (t, b) is stored at dest[b / bl][(b % bl) * t_out * d + table_slot[t] * d + k],
+ * bl = batch / n_dest, with the values dq_embbag_int4_fwd would give. Nothing else is
+ * written; the caller orders the ranks' calls against the reads of their buffers
+ * (a barrier after the calls, and one before the next call writes again).
+ * Errors: DQ_ERR_INVALID_ARG for the argument checks above (nothing launched).
+ */
+dq_status dq_embbag_int4_fwd_to_owners(const dq_table *tables, int32_t n_tables, int32_t d,
+                                       const int32_t *indices, const int32_t *offsets, int32_t batch,
+                                       const int32_t *table_slot, int32_t t_out, float *const *dest,
+                                       int32_t n_dest, uint32_t *d_flags, void *cuda_stream);
 
 /*
  * dq_row_l2_error -- normalized l2 error of packed rows against their binary32

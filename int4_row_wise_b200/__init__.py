@@ -28,7 +28,8 @@ __all__ = [
     "DQ_MODE_GREEDY", "DQ_MODE_MINMAX",
     "DQ_FLAG_BAD_INDEX", "DQ_FLAG_BAD_OFFSETS", "DQ_FLAG_NONFINITE", "DQ_FLAG_FP16_OVERFLOW",
     "DQ_MAX_D", "DQ_MAX_TABLES", "DqError", "PackedTable", "lib_path", "load",
-    "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_row_l2_error",
+    "dq_quantize_rows_int4", "dq_dequantize_rows", "dq_embbag_int4_fwd", "dq_embbag_int4_fwd_to_owners",
+    "dq_row_l2_error",
     "dq_embbag_int4_bwd_workspace_bytes", "dq_embbag_int4_bwd_sgd", "MasterTable",
     "dq_embbag_int4_bwd_sgd_noalloc", "DQ_BWD_STATIC_SCRATCH_BYTES",
     "dq_quantize_rows_kmeans4", "dq_dequantize_rows_kmeans4", "dq_embbag_kmeans4_fwd", "KmeansTable",
@@ -88,6 +89,8 @@ def load():
             L.dq_dequantize_rows.restype = ctypes.c_int
             L.dq_embbag_int4_fwd.argtypes = [vp, i32, i32, vp, vp, i32, vp, vp, vp]
             L.dq_embbag_int4_fwd.restype = ctypes.c_int
+            L.dq_embbag_int4_fwd_to_owners.argtypes = [vp, i32, i32, vp, vp, i32, vp, i32, vp, i32, vp, vp]
+            L.dq_embbag_int4_fwd_to_owners.restype = ctypes.c_int
             L.dq_row_l2_error.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, vp]
             L.dq_row_l2_error.restype = ctypes.c_int
             L.dq_embbag_int4_bwd_workspace_bytes.argtypes = [i32, i64]
@@ -185,9 +188,8 @@ class PackedTable(NamedTuple):
         return int(self.codes.shape[0])
 
 
-def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, out, d_flags=None,
-                       stream=None) -> None:
-    """C: dq_embbag_int4_fwd. tables: PackedTable (or (codes, scale_bias)) per table."""
+def _table_array(tables: Sequence):
+    """The dq_table array of PackedTable (or (codes, scale_bias)) entries."""
     arr = (_Table * max(len(tables), 1))()
     for t, tab in enumerate(tables):
         codes, sb = tab[0], tab[1]
@@ -196,9 +198,31 @@ def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, o
         # a table of 0 or 1 rows has no meaningful row stride: its row width is the stride
         ld = int(codes.stride(0)) if codes.shape[0] > 1 else int(codes.shape[1])
         arr[t] = _Table(_ptr(codes), _ptr(sb), int(codes.shape[0]), ld)
+    return arr
+
+
+def dq_embbag_int4_fwd(tables: Sequence, d: int, indices, offsets, batch: int, out, d_flags=None,
+                       stream=None) -> None:
+    """C: dq_embbag_int4_fwd. tables: PackedTable (or (codes, scale_bias)) per table."""
+    arr = _table_array(tables)
     st = load().dq_embbag_int4_fwd(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
                                    _ptr(offsets), batch, _ptr(out), _ptr(d_flags), _stream(stream))
     _check(st, "dq_embbag_int4_fwd")
+
+
+def dq_embbag_int4_fwd_to_owners(tables: Sequence, d: int, indices, offsets, batch: int, table_slot: Sequence[int],
+                                 t_out: int, dest: Sequence, d_flags=None, stream=None) -> None:
+    """C: dq_embbag_int4_fwd_to_owners. dest: one device buffer (tensor or address) per
+    rank, [batch // len(dest), t_out * d] binary32; table_slot: the column block of each
+    local table."""
+    arr = _table_array(tables)
+    slots = (ctypes.c_int32 * max(len(tables), 1))(*[int(v) for v in table_slot])
+    ptrs = (ctypes.c_void_p * max(len(dest), 1))(*[_ptr(x) for x in dest])
+    st = load().dq_embbag_int4_fwd_to_owners(ctypes.cast(arr, ctypes.c_void_p), len(tables), d, _ptr(indices),
+                                             _ptr(offsets), batch, ctypes.cast(slots, ctypes.c_void_p), t_out,
+                                             ctypes.cast(ptrs, ctypes.c_void_p), len(dest), _ptr(d_flags),
+                                             _stream(stream))
+    _check(st, "dq_embbag_int4_fwd_to_owners")
 
 
 class MasterTable(NamedTuple):

@@ -139,9 +139,10 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
     return launched(dq::launch_dequantize(a, sms, (cudaStream_t)cuda_stream), "dequantize");
 }
 
-dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d, const int32_t *indices,
-                             const int32_t *offsets, int32_t batch, float *out, uint32_t *d_flags,
-                             void *cuda_stream)
+namespace {
+
+// Checks and copies the lookup's tables (column block t of each output row by default).
+dq_status bag_tables(const dq_table *tables, int32_t n_tables, int32_t d, int32_t batch, dq::BagTables &tabs)
 {
     if (n_tables < 1 || n_tables > DQ_MAX_TABLES)
         return fail(DQ_ERR_INVALID_ARG, "n_tables = %d outside [1, %d]", n_tables, DQ_MAX_TABLES);
@@ -153,7 +154,6 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
         return fail(DQ_ERR_INVALID_ARG, "batch = %d < 0", batch);
     if ((int64_t)n_tables * batch + 1 > INT32_MAX)
         return fail(DQ_ERR_INVALID_ARG, "n_tables * batch + 1 offsets exceed int32 indexing");
-    dq::BagTables tabs;
     memset(&tabs, 0, sizeof tabs);
     for (int t = 0; t < n_tables; ++t) {
         const dq_table &tb = tables[t];
@@ -168,19 +168,102 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
         tabs.scale_bias[t] = tb.scale_bias;
         tabs.n_rows[t] = tb.n_rows;
         tabs.codes_ld[t] = tb.codes_ld;
+        tabs.slot[t] = t;
     }
-    if (batch > 0 && (!indices || !offsets || !out))
-        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
-    if (batch == 0)
-        return ok();
+    return DQ_OK;
+}
+
+dq_status bag_launch(const dq::BagTables &tabs, const dq::BagArgs &a, const dq::BagDest &dst, void *cuda_stream)
+{
     int sms = 0;
     dq_status st = current_device(&sms);
     if (st != DQ_OK)
         return st;
     if (fault_injected())
         return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
-    dq::BagArgs a{n_tables, d, batch, indices, offsets, out, d_flags, dq::make_batch_div((uint32_t)batch)};
-    return launched(dq::launch_embbag(tabs, a, sms, (cudaStream_t)cuda_stream), "embbag");
+    return launched(dq::launch_embbag(tabs, a, dst, sms, (cudaStream_t)cuda_stream), "embbag");
+}
+
+} // namespace
+
+dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d, const int32_t *indices,
+                             const int32_t *offsets, int32_t batch, float *out, uint32_t *d_flags,
+                             void *cuda_stream)
+{
+    dq::BagTables tabs;
+    dq_status st = bag_tables(tables, n_tables, d, batch, tabs);
+    if (st != DQ_OK)
+        return st;
+    if (batch > 0 && (!indices || !offsets || !out))
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
+    if (batch == 0)
+        return ok();
+    dq::BagArgs a{};
+    a.T = n_tables;
+    a.d = d;
+    a.batch = batch;
+    a.indices = indices;
+    a.offsets = offsets;
+    a.out = out;
+    a.flags = d_flags;
+    a.div = dq::make_batch_div((uint32_t)batch);
+    dq::BagDest dst{};   // n = 0: rows into out
+    return bag_launch(tabs, a, dst, cuda_stream);
+}
+
+dq_status dq_embbag_int4_fwd_to_owners(const dq_table *tables, int32_t n_tables, int32_t d,
+                                       const int32_t *indices, const int32_t *offsets, int32_t batch,
+                                       const int32_t *table_slot, int32_t t_out, float *const *dest,
+                                       int32_t n_dest, uint32_t *d_flags, void *cuda_stream)
+{
+    dq::BagTables tabs;
+    dq_status st = bag_tables(tables, n_tables, d, batch, tabs);
+    if (st != DQ_OK)
+        return st;
+    if (n_dest < 1 || n_dest > DQ_MAX_DEST)
+        return fail(DQ_ERR_INVALID_ARG, "n_dest = %d outside [1, %d]", n_dest, DQ_MAX_DEST);
+    if (batch % n_dest != 0)
+        return fail(DQ_ERR_INVALID_ARG, "batch = %d is not a multiple of n_dest = %d", batch, n_dest);
+    if (t_out < n_tables || (int64_t)t_out > (int64_t)DQ_MAX_TABLES * DQ_MAX_DEST)
+        return fail(DQ_ERR_INVALID_ARG, "t_out = %d outside [n_tables = %d, %d]", t_out, n_tables,
+                    DQ_MAX_TABLES * DQ_MAX_DEST);
+    if (!table_slot || !dest)
+        return fail(DQ_ERR_INVALID_ARG, "table_slot and dest must be non-NULL");
+    for (int t = 0; t < n_tables; ++t) {
+        if (table_slot[t] < 0 || table_slot[t] >= t_out)
+            return fail(DQ_ERR_INVALID_ARG, "table_slot[%d] = %d outside [0, %d)", t, table_slot[t], t_out);
+        for (int u = 0; u < t; ++u)
+            if (table_slot[u] == table_slot[t])
+                return fail(DQ_ERR_INVALID_ARG, "table_slot[%d] and table_slot[%d] are both %d", u, t,
+                            table_slot[t]);
+        tabs.slot[t] = table_slot[t];
+    }
+    if ((int64_t)(batch / n_dest) * t_out * d > ((int64_t)1 << 40))
+        return fail(DQ_ERR_INVALID_ARG, "the destination buffers exceed 2^40 elements");
+    if (batch > 0 && (!indices || !offsets))
+        return fail(DQ_ERR_INVALID_ARG, "indices and offsets must be non-NULL when batch > 0");
+    dq::BagDest dst{};
+    for (int r = 0; r < n_dest; ++r) {
+        if (batch > 0 && !dest[r])
+            return fail(DQ_ERR_INVALID_ARG, "dest[%d] must be non-NULL", r);
+        dst.ptr[r] = dest[r];
+    }
+    if (batch == 0)
+        return ok();
+    dq::BagArgs a{};
+    a.T = n_tables;
+    a.d = d;
+    a.batch = batch;
+    a.indices = indices;
+    a.offsets = offsets;
+    a.out = dest[0];   // not written: every row goes through dst
+    a.flags = d_flags;
+    a.div = dq::make_batch_div((uint32_t)batch);
+    dst.n = n_dest;
+    dst.bl = batch / n_dest;
+    dst.t_out = t_out;
+    dst.div = dq::make_batch_div((uint32_t)dst.bl);
+    return bag_launch(tabs, a, dst, cuda_stream);
 }
 
 dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, const uint8_t *codes,

@@ -324,9 +324,9 @@ __device__ __forceinline__ void clamp_bag(int32_t &p, int32_t &p1, int32_t n_ids
 }
 
 // Long bags: IS id strides per element group, reduce-scatter, contiguous row stores.
-template <int E, int IS>
-__device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagArgs &a, uint32_t total,
-                                               int32_t n_ids)
+template <int E, int IS, class D>
+__device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagArgs &a, const D &dst,
+                                               uint32_t total, int32_t n_ids)
 {
     const int EG = a.d / E;
     const int G = EG * IS;     // lanes per bag, a power of two <= 32
@@ -366,7 +366,7 @@ __device__ __forceinline__ void bag_tiles_long(const BagTables &tabs, const BagA
         reduce_scatter<E, IS>(acc, is);
         if (live) {
             constexpr int C = E / IS;  // finished sums owned by this lane
-            float *o = a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d + eg * E + is * C;
+            float *o = bag_row(tabs, a, dst, t, b) + eg * E + is * C;
             if constexpr (C % 4 == 0) {
 #pragma unroll
                 for (int k = 0; k < C; k += 4)
@@ -480,9 +480,9 @@ struct OnehotSlot {
 // store writes 32 / LB whole rows; the loads of UNR sub-steps are issued before any is
 // decoded, and a one-id bag's row is fma(q, scale, bias) written directly (no sum).
 // Bags with two or more ids are then summed one at a time by the warp's first LB lanes.
-template <int EL>
-__device__ __forceinline__ void bag_tiles_onehot(const BagTables &tabs, const BagArgs &a, uint32_t total,
-                                                 int32_t n_ids, OnehotSlot *slots)
+template <int EL, class D>
+__device__ __forceinline__ void bag_tiles_onehot(const BagTables &tabs, const BagArgs &a, const D &dst,
+                                                 uint32_t total, int32_t n_ids, OnehotSlot *slots)
 {
     using CV = typename ChunkVec<EL>::T;
     constexpr unsigned FULL = 0xffffffffu;
@@ -509,7 +509,7 @@ __device__ __forceinline__ void bag_tiles_onehot(const BagTables &tabs, const Ba
             clamp_bag(p, p1, n_ids, true, a.flags);
             const int t = (int)div_batch((uint32_t)g, a.div);
             const int b = (int)((uint32_t)g - (uint32_t)t * batch);
-            sl.out = a.out + ((int64_t)b * a.T + t) * a.d;
+            sl.out = bag_row(tabs, a, dst, t, b);
             if (p1 == p + 1) {
                 const uint32_t id = (int64_t)p == (int64_t)g ? (uint32_t)cur.id : (uint32_t)__ldg(a.indices + p);
                 if ((int64_t)id < tabs.n_rows[t]) {
@@ -615,22 +615,23 @@ __device__ __forceinline__ void bag_tiles_onehot(const BagTables &tabs, const Ba
 // E1: elements per lane chunk of the one-hot layout; E, ISL: elements per lane and
 // id strides of the long layout. The kernel reads the id count (the last offset) and
 // takes the long layout when bags average 4 ids or more.
-template <int E1, int E, int ISL>
+template <int E1, int E, int ISL, class D>
 __global__ void __launch_bounds__(kBagThreads, E == 16 ? 4 : 1) embbag_kernel(const __grid_constant__ BagTables tabs,
-                                                                             const BagArgs a)
+                                                                             const BagArgs a,
+                                                                             const __grid_constant__ D dst)
 {
     __shared__ __align__(16) OnehotSlot slots[kBagThreads / 32][32];
     const int64_t total = (int64_t)a.T * a.batch;
     const int32_t n_ids = max(__ldg(a.offsets + total), 0);
     if (ISL > 1 && (int64_t)n_ids >= 4 * total)   // average pooling >= 4: split ids over lanes
-        bag_tiles_long<E, ISL>(tabs, a, (uint32_t)total, n_ids);
+        bag_tiles_long<E, ISL>(tabs, a, dst, (uint32_t)total, n_ids);
     else
-        bag_tiles_onehot<E1>(tabs, a, (uint32_t)total, n_ids, slots[threadIdx.x >> 5]);
+        bag_tiles_onehot<E1>(tabs, a, dst, (uint32_t)total, n_ids, slots[threadIdx.x >> 5]);
 }
 
 // any d, any alignment: one warp per bag, lanes stride over the elements
 __global__ void __launch_bounds__(256) embbag_generic_kernel(const __grid_constant__ BagTables tabs,
-                                                             const BagArgs a)
+                                                             const BagArgs a, const __grid_constant__ BagDest dst)
 {
     const int64_t total = (int64_t)a.T * a.batch;
     const int lane = threadIdx.x & 31;
@@ -647,7 +648,7 @@ __global__ void __launch_bounds__(256) embbag_generic_kernel(const __grid_consta
         p0 = min(max(p0, 0), n_ids);
         p1 = max(min(p1, n_ids), p0);
     }
-    float *o = a.out + (int64_t)b * a.T * a.d + (int64_t)t * a.d;
+    float *o = bag_row(tabs, a, dst, t, b);
     const int64_t n_rows = tabs.n_rows[t];
     for (int k0 = 0; k0 < a.d; k0 += 32) {
         const int k = k0 + lane;
@@ -671,6 +672,24 @@ __global__ void __launch_bounds__(256) embbag_generic_kernel(const __grid_consta
         if (k < a.d)
             o[k] = acc;
     }
+}
+
+// D: BagDest (rows into the owners' buffers) or NoDest (rows into out). Separate
+// instantiations, so that the plain lookup's parameters and registers stay as they are.
+template <class D>
+void launch_fast(const BagTables &tabs, const BagArgs &a, const D &dst, int E, int isl, unsigned grid,
+                 cudaStream_t stream)
+{
+    if (E == 32)
+        embbag_kernel<32, 32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a, dst);   // d = 1024
+    else if (isl == 8)
+        embbag_kernel<4, 16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a, dst);    // d = 16, 32, 64
+    else if (isl == 4)
+        embbag_kernel<4, 16, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a, dst);    // d = 128
+    else if (isl == 2)
+        embbag_kernel<8, 16, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a, dst);    // d = 256
+    else
+        embbag_kernel<16, 16, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a, dst);   // d = 512
 }
 
 int grid_for(int64_t work, int block, int num_sms)
@@ -699,7 +718,8 @@ cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t st
     return cudaGetLastError();
 }
 
-cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream)
+cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, const BagDest &dst, int num_sms,
+                          cudaStream_t stream)
 {
     const int64_t total = (int64_t)a.T * a.batch;
     int E = 0;
@@ -708,6 +728,8 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, 
     else if (a.d % 32 == 0 && a.d / 32 <= 32 && ((a.d / 32) & (a.d / 32 - 1)) == 0)
         E = 32;
     bool fast = E != 0 && (reinterpret_cast<uintptr_t>(a.out) & 15) == 0;
+    for (int r = 0; fast && r < dst.n; ++r)   // rows stored into the owners' buffers
+        fast = (reinterpret_cast<uintptr_t>(dst.ptr[r]) & 15) == 0;
     for (int t = 0; fast && t < a.T; ++t)
         fast = tabs.codes_ld[t] % (E / 2) == 0 && (reinterpret_cast<uintptr_t>(tabs.codes[t]) % (E / 2)) == 0 &&
                (reinterpret_cast<uintptr_t>(tabs.scale_bias[t]) & 3) == 0;
@@ -719,19 +741,13 @@ cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, 
         const int64_t need = long_tiles > onehot_blocks ? long_tiles : onehot_blocks;
         const int64_t cap = (int64_t)num_sms * 8;
         const unsigned grid = (unsigned)(need < cap ? need : cap);
-        if (E == 32)
-            embbag_kernel<32, 32, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);   // d = 1024
-        else if (isl == 8)
-            embbag_kernel<4, 16, 8><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 16, 32, 64
-        else if (isl == 4)
-            embbag_kernel<4, 16, 4><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 128
-        else if (isl == 2)
-            embbag_kernel<8, 16, 2><<<grid, kBagThreads, 0, stream>>>(tabs, a);    // d = 256
+        if (dst.n > 0)
+            launch_fast(tabs, a, dst, E, isl, grid, stream);
         else
-            embbag_kernel<16, 16, 1><<<grid, kBagThreads, 0, stream>>>(tabs, a);   // d = 512
+            launch_fast(tabs, a, NoDest{0}, E, isl, grid, stream);
     } else {
         const int64_t grid = (total * 32 + 255) / 256;
-        embbag_generic_kernel<<<(unsigned)grid, 256, 0, stream>>>(tabs, a);
+        embbag_generic_kernel<<<(unsigned)grid, 256, 0, stream>>>(tabs, a, dst);
     }
     return cudaGetLastError();
 }

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "dq.h"
 
 namespace dq {
@@ -39,6 +41,7 @@ struct BagTables {
     const uint16_t *scale_bias[DQ_MAX_TABLES];
     int64_t n_rows[DQ_MAX_TABLES];
     int64_t codes_ld[DQ_MAX_TABLES];
+    int32_t slot[DQ_MAX_TABLES];   // the table's column block in the output rows
 };
 
 struct L2Args {
@@ -66,6 +69,15 @@ struct BagArgs {
     float *out;
     uint32_t *flags;
     BatchDiv div;
+};
+
+// Where bag (t, b) is stored: with n == 0, out[b][t*d ..]; otherwise the row of sample
+// b % bl in ptr[b / bl], column block slot[t] of t_out. A kernel parameter of its own:
+// folded into BagArgs it made the 64-register lookup kernels spill.
+struct BagDest {
+    int n, bl, t_out;
+    BatchDiv div;
+    float *ptr[DQ_MAX_DEST];
 };
 
 // Master and packed tables of the bag backward, passed by value (about 2.8 KB of
@@ -179,9 +191,29 @@ __device__ __forceinline__ uint32_t div_batch(uint32_t n, const BatchDiv &v)
     return (t + ((n - t) >> v.sh1)) >> v.sh2;
 }
 
+// The output row of bag (t, b) of a lookup (see BagArgs).
+// The plain lookup's kernels take this in place of BagDest (rows go to out).
+struct NoDest {
+    int n;
+};
+
+template <class D>
+__device__ __forceinline__ float *bag_row(const BagTables &tabs, const BagArgs &a, const D &dst, int t, int b)
+{
+    if constexpr (std::is_same<D, BagDest>::value) {
+        if (dst.n > 0) {
+            const uint32_t r = div_batch((uint32_t)b, dst.div);
+            const int64_t s = (int64_t)b - (int64_t)r * dst.bl;
+            return dst.ptr[r] + (s * dst.t_out + tabs.slot[t]) * a.d;
+        }
+    }
+    return a.out + ((int64_t)b * a.T + t) * a.d;
+}
+
 cudaError_t launch_quantize(const QuantArgs &a, int mode, int num_sms, cudaStream_t stream);
 cudaError_t launch_dequantize(const DequantArgs &a, int num_sms, cudaStream_t stream);
-cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, int num_sms, cudaStream_t stream);
+cudaError_t launch_embbag(const BagTables &tabs, const BagArgs &a, const BagDest &dst, int num_sms,
+                          cudaStream_t stream);
 cudaError_t launch_row_l2(const L2Args &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_bwd_sort_reduce(BwdArgs &a, int num_sms, cudaStream_t stream);
 cudaError_t launch_kmeans(const KmeansArgs &a, cudaStream_t stream);

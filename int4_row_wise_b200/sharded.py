@@ -14,12 +14,19 @@ Host synchronisation: sharded_embbag needs none; sharded_embbag_local reads two 
 count arrays back to the host (the all-to-all split sizes must be host integers):
 every table's first and last offset before the exchange, and the received per-(source,
 table) id counts after the bag lengths have been exchanged.
+
+Direct form (OwnerBuffers): every rank maps all ranks' receive buffers into its address
+space (CUDA IPC through torch's storage sharing) and one kernel,
+dq_embbag_int4_fwd_to_owners, stores each pooled row straight into its owner's buffer
+at its final place: no all-to-all, no reassembly copy. The ranks meet at a barrier
+before each call (the owners have read the previous result) and after it (every row
+has arrived).
 """
 from __future__ import annotations
 
 from typing import Callable, List, Optional, Sequence
 
-__all__ = ["plan_tables", "sharded_embbag", "sharded_embbag_local"]
+__all__ = ["plan_tables", "sharded_embbag", "sharded_embbag_local", "OwnerBuffers", "sharded_embbag_direct"]
 
 
 def plan_tables(rows: Sequence[int], world: int) -> List[int]:
@@ -179,3 +186,77 @@ def sharded_embbag_local(local_tables: Sequence, owner: Sequence[int], d: int, b
     offsets[1:] = torch.cumsum(lens.permute(1, 0, 2).reshape(-1), dim=0).to(torch.int32)
     return sharded_embbag(local_tables, owner, d, indices, offsets, world * local_batch, group=group,
                           lookup=lookup)
+
+
+class OwnerBuffers:
+    """Every rank's receive buffer [batch // world, T * d] binary32, as device addresses
+    usable by this rank's kernels: this rank's own tensor, and the others' buffers opened
+    from the CUDA IPC handles of their storages (exchanged once, at creation)."""
+
+    def __init__(self, own, addresses: List[int], keep: list):
+        self.own = own                # this rank's buffer (the rows it owns)
+        self.addresses = addresses    # device address of rank r's buffer, r = 0 .. world-1
+        self._keep = keep             # the opened storages of the other ranks
+
+    @classmethod
+    def create(cls, local_batch: int, width: int, device, group=None) -> "OwnerBuffers":
+        import torch
+        import torch.distributed as dist
+        own = torch.zeros((local_batch, width), dtype=torch.float32, device=device)
+        world = dist.get_world_size(group) if dist.is_initialized() else 1
+        if world == 1:
+            return cls(own, [own.data_ptr()], [])
+        rank = dist.get_rank(group)
+        storage = own.untyped_storage()
+        handles = [None] * world
+        dist.all_gather_object(handles, (storage._share_cuda_(), own.storage_offset() * own.element_size()),
+                               group=group)
+        addresses, keep = [], []
+        for r, (h, off) in enumerate(handles):
+            if r == rank:
+                addresses.append(own.data_ptr())
+                continue
+            peer = torch.UntypedStorage._new_shared_cuda(*h)
+            keep.append(peer)
+            addresses.append(peer.data_ptr() + off)
+        return cls(own, addresses, keep)
+
+
+def sharded_embbag_direct(local_tables: Sequence, owner: Sequence[int], d: int, indices, offsets, global_batch: int,
+                          buffers: OwnerBuffers, group=None):
+    """sharded_embbag with the exchange folded into the lookup: this rank's tables' rows
+    for the global batch are stored straight into the owners' buffers (buffers.addresses,
+    one per rank, each [global_batch // world, T * d]) at the column block of their global
+    table. Returns this rank's buffer (the rows of its samples, all tables) once every
+    rank's rows have arrived."""
+    import torch
+    import torch.distributed as dist
+    import int4_row_wise_b200 as dq
+
+    world = dist.get_world_size(group) if dist.is_initialized() else 1
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
+    _check_owner(owner, world)
+    if global_batch % world:
+        raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
+    if len(buffers.addresses) != world:
+        raise ValueError(f"{len(buffers.addresses)} owner buffers for {world} ranks")
+    T = len(owner)
+    if tuple(buffers.own.shape) != (global_batch // world, T * d):
+        raise ValueError(f"own buffer {tuple(buffers.own.shape)}, expected {(global_batch // world, T * d)}")
+    mine = [t for t, r in enumerate(owner) if r == rank]
+    if len(mine) != len(local_tables):
+        raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
+    if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
+        raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x {global_batch} bags "
+                         f"need {len(mine) * global_batch + 1}")
+    stream = torch.cuda.current_stream(buffers.own.device)
+    if world > 1:   # the owners have read the previous result
+        stream.synchronize()
+        dist.barrier(group)
+    if mine:
+        dq.dq_embbag_int4_fwd_to_owners(local_tables, d, indices, offsets, global_batch, mine, T,
+                                        buffers.addresses, None, stream)
+    if world > 1:   # every rank's rows have arrived
+        stream.synchronize()
+        dist.barrier(group)
+    return buffers.own

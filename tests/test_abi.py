@@ -100,6 +100,27 @@ def test_embbag_rejects(L, tabspec, T, d, batch, msg):
     assert msg in L.dq_last_error().decode()
 
 
+@pytest.mark.parametrize("batch,slots,t_out,n_dest,msg", [
+    (6, [0], 1, 4, "not a multiple"),
+    (4, [0], 1, 0, "n_dest = 0"),
+    (4, [0], 1, 65, "n_dest = 65"),
+    (4, [1], 1, 2, "table_slot[0] = 1"),
+    (4, [-1], 3, 2, "table_slot[0] = -1"),
+    (4, [0, 0], 3, 2, "both 0"),
+    (4, [0, 1], 1, 2, "t_out = 1"),
+])
+def test_embbag_to_owners_rejects(L, batch, slots, t_out, n_dest, msg):
+    """The placement checks come before anything touches a GPU."""
+    T = len(slots)
+    p, keep = _tables(*[(1 << 20, 1 << 21, 10, 8)] * T)
+    sl = (ctypes.c_int32 * T)(*slots)
+    dest = (ctypes.c_void_p * max(n_dest, 1))(*([1 << 24] * max(n_dest, 1)))
+    st = L.dq_embbag_int4_fwd_to_owners(p, T, 16, 1 << 22, 1 << 23, batch, ctypes.cast(sl, ctypes.c_void_p), t_out,
+                                        ctypes.cast(dest, ctypes.c_void_p), n_dest, None, None)
+    assert st == dq.DQ_ERR_INVALID_ARG
+    assert msg in L.dq_last_error().decode()
+
+
 def test_binding_raises_with_status(L):
     with pytest.raises(dq.DqError) as ei:
         dq.dq_quantize_rows_int4(None, 4, 0, 16, None, 8, None, stream=0)

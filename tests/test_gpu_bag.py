@@ -114,6 +114,38 @@ def test_bag_rows_of_every_scale(cuda_device, d):
         assert np.array_equal(got[one].view(np.uint32), ref[one].view(np.uint32))
 
 
+@pytest.mark.parametrize("n_dest", [1, 2, 3, 4])
+@pytest.mark.parametrize("d,pool", [(16, (1, 1)), (64, (4, 12)), (128, (0, 3)), (100, (1, 6))])
+def test_bag_to_owners_matches_oracle(cuda_device, n_dest, d, pool):
+    """dq_embbag_int4_fwd_to_owners over n_dest buffers on one GPU: bag (t, b) lands in
+    buffer b // bl, row b % bl, column block slot[t] of t_out, with the lookup's values;
+    the other column blocks are left as they were."""
+    T, B, t_out = 3, 96, 5
+    slots = [4, 0, 2]
+    rows = [500, 1000, 37]
+    cld = ((d + 1) // 2 + 15) // 16 * 16
+    tabs = [_packed(n, d, 30 * d + t, cld) for t, n in enumerate(rows)]
+    idx, off = _bags(T, B, rows, pool[0], pool[1], d + n_dest)
+    ref, mag, _ = oracle.embbag(tabs, d, idx, off, B, with_abs_sum=True)
+    bl = B // n_dest
+    dest = [torch.full((bl, t_out * d), 7.0, dtype=torch.float32, device="cuda") for _ in range(n_dest)]
+    dev_tabs = [dq.PackedTable(to_dev(c), to_dev(s.view(np.int16))) for c, s in tabs]
+    dq.dq_embbag_int4_fwd_to_owners(dev_tabs, d, to_dev(idx if idx.size else np.zeros(1, np.int32)), to_dev(off), B,
+                                    slots, t_out, dest)
+    torch.cuda.synchronize()
+    got = np.empty((B, T * d), np.float32)
+    for r in range(n_dest):
+        o = dest[r].cpu().numpy()
+        for t, sl in enumerate(slots):
+            got[r * bl:(r + 1) * bl, t * d:(t + 1) * d] = o[:, sl * d:(sl + 1) * d]
+        for sl in set(range(t_out)) - set(slots):
+            assert np.all(o[:, sl * d:(sl + 1) * d] == 7.0)
+    bag_tolerance_check(got, ref, mag)
+    lens = np.diff(off.astype(np.int64)).reshape(T, B).T
+    one = np.repeat(lens == 1, d, axis=1)
+    assert np.array_equal(got[one].view(np.uint32), ref[one].view(np.uint32))
+
+
 def test_bag_bad_ids_and_offsets(cuda_device):
     d, T, B = 64, 2, 50
     rows = [100, 100]

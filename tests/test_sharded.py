@@ -141,7 +141,12 @@ def test_sharded_lookup_on_the_gpu_against_the_oracle(nccl_one_rank, d, pool):
     ref, mag, _ = oracle.embbag(tables, d, idx, off, B, with_abs_sum=True)
     lens = np.stack([o[1:] - o[:-1] for _, o in per_table], axis=1)          # [B, T]
     one = np.repeat(lens == 1, d, axis=1)                                      # elements of one-id bags
-    for out in (got, routed):
+    # the direct form: the lookup stores every row straight into its owner's buffer
+    from int4_row_wise_b200.sharded import OwnerBuffers, sharded_embbag_direct
+    bufs = OwnerBuffers.create(B, T * d, torch.device("cuda", 0))
+    direct = sharded_embbag_direct(dt, owner, d, torch.from_numpy(idx).cuda(), torch.from_numpy(off).cuda(), B, bufs)
+    torch.cuda.synchronize()
+    for out in (got, routed, direct):
         o = out.cpu().numpy()
         bag_tolerance_check(o, ref, mag)
         assert np.array_equal(o[one].view(np.uint32), ref[one].view(np.uint32))
