@@ -65,10 +65,10 @@ OTHER_WORKLOADS = ("tiny", "kaggle", "terabyte", "sweep-16", "sweep-32", "sweep-
 # quantizer (`ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum -k regex:quantize_rows
 # -s 3 -c 1` around `bench.py --workload W --steps 1 --warmup 3 --no-per-workload --no-e2e
 # --no-cpu-baseline --no-next-rows`): d=16, a Kaggle-shaped table of 3,097,041 rows, 199.1 MB
-# read + 25.9 MB written; d=128, the sweep d=128 table of 1,000,000 rows, 514.8 MB read +
-# 61.5 MB written. A launch's traffic scales with its rows at a fixed d; it is reported only
+# read + 25.6 MB written; d=128, the sweep d=128 table of 1,000,000 rows, 514.8 MB read +
+# 61.6 MB written. A launch's traffic scales with its rows at a fixed d; it is reported only
 # for a captured d and while the kernel source still has the recorded sha256 prefix.
-NCU_QUANT_TRAFFIC = {"kernel_sha": "76c38611eb740cec", "bytes_per_row": {16: 72.65, 128: 576.29}}
+NCU_QUANT_TRAFFIC = {"kernel_sha": "b1b4606e303e4827", "bytes_per_row": {16: 72.56, 128: 576.39}}
 
 
 # ---------------------------------------------------------------------------
