@@ -651,6 +651,18 @@ def _workload_entry(args, wl: W.Workload, dev, dq) -> dict:
     return entry
 
 
+def _kmeans_ops(d: int, iters: int, row_iters) -> tuple:
+    """ALU ops the codebook quantizer executed over rows whose per-row Lloyd iteration
+    counts (the kernel's row_iters output) are given: per element and centroid update 16
+    distances (subtract, compare) and one add into its own cluster (33); the assignment
+    that found the repeat (32) for rows that stopped early; the final 16 distances and the
+    loss terms (35). Returns (ops, centroid updates run per row)."""
+    ran = sum(int(r.sum()) for r in row_iters)
+    stopped = sum(int((r < iters).sum()) for r in row_iters)
+    rows = sum(int(r.numel()) for r in row_iters)
+    return float(d) * (33 * ran + 32 * stopped + 35 * rows), ran / max(rows, 1)
+
+
 def _next_rows(wl, xs, step, dev, dq) -> dict:
     """The codebook quantizer (all tables, 3 steps, then one codebook lookup per step) and
     the bag backward + SGD + re-quantization (10 calls over the step's lookup batches,
@@ -667,13 +679,15 @@ def _next_rows(wl, xs, step, dev, dq) -> dict:
     kc = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wl.rows]
     kcb = [torch.empty((n, 16), dtype=torch.int16, device=dev) for n in wl.rows]
     kt = [dq.KmeansTable(c, b) for c, b in zip(kc, kcb)]
+    kit = [torch.empty(n, dtype=torch.int32, device=dev) for n in wl.rows]
     bag_out = torch.empty((B, T * d), dtype=torch.float32, device=dev)
     iters = dq.KMEANS_ITERS
 
     def cb_step(k):
         for t, x in enumerate(xs):
             if wl.rows[t]:
-                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, kc[t], cld, kcb[t], None, iters, None, stream)
+                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, kc[t], cld, kcb[t], None, iters, None, stream,
+                                            row_iters=kit[t])
         i, o = step.batches[k % len(step.batches)]
         dq.dq_embbag_kmeans4_fwd(kt, d, i, o, B, bag_out, None, stream)
 
@@ -692,17 +706,18 @@ def _next_rows(wl, xs, step, dev, dq) -> dict:
     xu = dq.dequantize_rows(step.codes[t][:n_q], step.sbs[t][:n_q], d).double()
     nrm = x64.norm(dim=1)
     ok = nrm > 0
-    cb_flops = wl.total_rows * d * (iters * 33 + 35)
+    cb_flops, cb_iters_run = _kmeans_ops(d, iters, [r for r, n in zip(kit, wl.rows) if n])
     cb_peak = FP32_LANES_PER_SM * sms * SM_MHZ_MAX * 1e6 / 1e12
     out["codebook"] = {
         "what": "codebook 4-bit quantization (per-row k-means, 16 binary16 centroids, "
                 f"{iters} Lloyd iterations) of all tables + one codebook lookup call",
         "rows_per_s": wl.total_rows / (cb_ms / 1e3), "ms_per_step": cb_ms,
+        "lloyd_updates_run_per_row": cb_iters_run,
         "alu_frac_upper": cb_flops / (cb_ms / 1e3) / 1e12 / cb_peak, "alu_peak_tops": cb_peak,
         "normalized_l2_codebook": float(((x64 - xk).norm(dim=1)[ok] / nrm[ok]).mean()),
         "normalized_l2_greedy": float(((x64 - xu).norm(dim=1)[ok] / nrm[ok]).mean()),
         "bytes_per_row": {"codebook": (d + 1) // 2 + 32, "greedy": (d + 1) // 2 + 4}}
-    del kc, kcb, kt, xk, xu, x64
+    del kc, kcb, kt, kit, xk, xu, x64
     torch.cuda.empty_cache()
     gen = torch.Generator(device=dev)
     gen.manual_seed(4321)
@@ -1018,6 +1033,7 @@ def run_codebook(args, wl: W.Workload) -> None:
     codes = [torch.empty((n, cld), dtype=torch.uint8, device=dev) for n in wl.rows]
     cbs = [torch.empty((n, 16), dtype=torch.int16, device=dev) for n in wl.rows]
     tables = [dq.KmeansTable(c, b) for c, b in zip(codes, cbs)]
+    its = [torch.empty(n, dtype=torch.int32, device=dev) for n in wl.rows]
     n_batches = 4
     bh = [W.lookup_batch(wl, batch_id=i) for i in range(n_batches)]
     bd = [(torch.from_numpy(i).to(dev), torch.from_numpy(o).to(dev)) for i, o in bh]
@@ -1030,7 +1046,8 @@ def run_codebook(args, wl: W.Workload) -> None:
             ev[0].record(stream)
         for t, x in enumerate(xs):
             if wl.rows[t]:
-                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, codes[t], cld, cbs[t], None, iters, None, stream)
+                dq.dq_quantize_rows_kmeans4(x, wl.rows[t], d, d, codes[t], cld, cbs[t], None, iters, None, stream,
+                                            row_iters=its[t])
         if ev:
             ev[1].record(stream)
         i, o = bd[k % n_batches]
@@ -1050,9 +1067,10 @@ def run_codebook(args, wl: W.Workload) -> None:
     q_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     tot_ms = sum(e[0].elapsed_time(e[2]) for e in evs)
     rows = wl.total_rows * args.steps
-    # algorithmic work per element: per iteration 16 distances (subtract, compare) and one
-    # add into the element's own cluster; then the final 16 distances and the loss terms
-    flops = wl.total_rows * d * (iters * 33 + 35) * args.steps
+    # ALU work the kernel executed (every step quantizes the same tables: the same
+    # iteration counts)
+    ops_step, iters_run = _kmeans_ops(d, iters, [r for r, n in zip(its, wl.rows) if n])
+    flops = ops_step * args.steps
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     peak = FP32_LANES_PER_SM * sms * SM_MHZ_MAX * 1e6 / 1e12  # one FP32 op per lane per clock (no FMA here)
     achieved = flops / (q_ms / 1e3) / 1e12
@@ -1076,7 +1094,9 @@ def run_codebook(args, wl: W.Workload) -> None:
         "config": {"workload": _workload_desc(wl), "lloyd_iterations": iters},
         "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                      "peak_source": f"{FP32_LANES_PER_SM} FP32 lanes x {sms} SMs x 1965 MHz, one op per lane-clock",
-                     "flops_per_element": iters * 33 + 35},
+                     "ops_per_element": "33 per centroid update run + 32 for the repeat check of a row that "
+                                        "stopped early + 35 (final assignment and loss)",
+                     "lloyd_updates_run_per_row": iters_run},
         "embbag": _brief(bag),
         "quality": {"normalized_l2_codebook": l2k, "normalized_l2_greedy_uniform": l2u, "rows": n_q,
                     "bytes_per_row_codebook": rb, "bytes_per_row_uniform": (d + 1) // 2 + 4},

@@ -219,11 +219,16 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
 
 /* dq_quantize_rows_kmeans4 -- arguments as dq_quantize_rows_int4, with codebook
  * [n_rows][16] binary16 (output, 2-byte aligned), row_loss [n_rows] (nullable), iters in
- * [0, DQ_KMEANS_MAX_ITERS]; d_flags: DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW. */
+ * [0, DQ_KMEANS_MAX_ITERS]; d_flags: DQ_FLAG_NONFINITE, DQ_FLAG_FP16_OVERFLOW.
+ * Once an iteration's assignment q equals the previous iteration's, the centroids it
+ * would compute are the current ones, so every later iteration repeats them: the
+ * library stops there (the outputs are those of all `iters` iterations). row_iters
+ * [n_rows] (int32, nullable, device): the centroid updates run for each row, at most
+ * iters (rows processed together run until all of them have repeated). */
 dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld,
                                    uint8_t *codes, int64_t codes_ld, uint16_t *codebook,
-                                   float *row_loss, int32_t iters, uint32_t *d_flags,
-                                   void *cuda_stream);
+                                   float *row_loss, int32_t *row_iters, int32_t iters,
+                                   uint32_t *d_flags, void *cuda_stream);
 
 /* dq_dequantize_rows_kmeans4 -- out[r][k] = codebook[r][q_k] (exact). */
 dq_status dq_dequantize_rows_kmeans4(const uint8_t *codes, int64_t codes_ld,

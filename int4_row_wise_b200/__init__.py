@@ -101,7 +101,7 @@ def load():
             L.dq_embbag_int4_bwd_sgd_noalloc.argtypes = [vp, i32, i32, vp, vp, i32, i64, vp, ctypes.c_float, i32,
                                                          vp, vp]
             L.dq_embbag_int4_bwd_sgd_noalloc.restype = ctypes.c_int
-            L.dq_quantize_rows_kmeans4.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, i32, vp, vp]
+            L.dq_quantize_rows_kmeans4.argtypes = [vp, i64, i32, i64, vp, i64, vp, vp, vp, i32, vp, vp]
             L.dq_quantize_rows_kmeans4.restype = ctypes.c_int
             L.dq_dequantize_rows_kmeans4.argtypes = [vp, i64, vp, i64, i32, vp, i64, vp]
             L.dq_dequantize_rows_kmeans4.restype = ctypes.c_int
@@ -272,10 +272,10 @@ class KmeansTable(NamedTuple):
 
 
 def dq_quantize_rows_kmeans4(x, n_rows: int, d: int, x_ld: int, codes, codes_ld: int, codebook, row_loss=None,
-                             iters: int = KMEANS_ITERS, d_flags=None, stream=None) -> None:
-    """C: dq_quantize_rows_kmeans4."""
+                             iters: int = KMEANS_ITERS, d_flags=None, stream=None, row_iters=None) -> None:
+    """C: dq_quantize_rows_kmeans4 (row_iters: optional int32 [n_rows] device tensor)."""
     st = load().dq_quantize_rows_kmeans4(_ptr(x), n_rows, d, x_ld, _ptr(codes), codes_ld, _ptr(codebook),
-                                         _ptr(row_loss), iters, _ptr(d_flags), _stream(stream))
+                                         _ptr(row_loss), _ptr(row_iters), iters, _ptr(d_flags), _stream(stream))
     _check(st, "dq_quantize_rows_kmeans4")
 
 

@@ -295,8 +295,8 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
 }
 
 dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, int64_t x_ld, uint8_t *codes,
-                                   int64_t codes_ld, uint16_t *codebook, float *row_loss, int32_t iters,
-                                   uint32_t *d_flags, void *cuda_stream)
+                                   int64_t codes_ld, uint16_t *codebook, float *row_loss, int32_t *row_iters,
+                                   int32_t iters, uint32_t *d_flags, void *cuda_stream)
 {
     if (n_rows < 0)
         return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld < 0", (long long)n_rows);
@@ -320,7 +320,7 @@ dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, in
         return st;
     if (fault_injected())
         return fail(DQ_ERR_CUDA, "launch failure injected by DQ_FAULT_INJECT=launch");
-    dq::KmeansArgs a{x, n_rows, x_ld, d, iters, codes, codes_ld, codebook, row_loss, d_flags};
+    dq::KmeansArgs a{x, n_rows, x_ld, d, iters, codes, codes_ld, codebook, row_loss, row_iters, d_flags};
     return launched(dq::launch_kmeans(a, (cudaStream_t)cuda_stream), "quantize_rows_kmeans4");
 }
 

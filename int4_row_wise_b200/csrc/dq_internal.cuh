@@ -137,6 +137,7 @@ struct KmeansArgs {
     int64_t codes_ld;
     uint16_t *codebook;        // [n][16] binary16
     float *row_loss;
+    int32_t *row_iters;        // [n], nullable: Lloyd iterations run for the row
     uint32_t *flags;
 };
 

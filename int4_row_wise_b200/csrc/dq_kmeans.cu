@@ -17,7 +17,8 @@
 // builds the tree of its aligned block bottom-up, and an XOR butterfly over the W
 // lanes joins the blocks in tree order; IEEE addition is commutative, so every lane
 // of a row ends with the identical sums and centroids. ALU bound: each iteration
-// costs 16 distance evaluations and 16 masked adds per element.
+// costs 16 distance evaluations and 16 masked adds per element. A warp stops iterating
+// once every row's assignment has repeated (a fixed point of the iteration).
 #include <cfloat>
 
 #include "dq_internal.cuh"
@@ -174,10 +175,34 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
             c[j] = __fmaf_rn((float)j, step, mn);
     }
     __syncwarp();
-    // K2: Lloyd iterations
+    // K2: Lloyd iterations. When an assignment repeats the previous one, the update would
+    // reproduce the current centroids, and so would every later iteration: the warp stops
+    // once all its rows have repeated (rows that repeated earlier recompute their own
+    // centroids unchanged until then).
     uint8_t q[M];
-    for (int it = 0; it < a.iters; ++it) {
+    constexpr int kWords = (M + 7) / 8;  // the lane's codes, 4 bits each
+    uint32_t prev[kWords];
+#pragma unroll
+    for (int w = 0; w < kWords; ++w)
+        prev[w] = 0u;
+    int it = 0;
+    for (; it < a.iters; ++it) {
         nearest<M>(x, c, q);
+        uint32_t pk[kWords];
+#pragma unroll
+        for (int w = 0; w < kWords; ++w)
+            pk[w] = 0u;
+#pragma unroll
+        for (int m = 0; m < M; ++m)
+            pk[m / 8] |= (uint32_t)q[m] << (4 * (m % 8));
+        bool same = it > 0;
+#pragma unroll
+        for (int w = 0; w < kWords; ++w) {
+            same &= pk[w] == prev[w];
+            prev[w] = pk[w];
+        }
+        if (__all_sync(0xffffffffu, same))
+            break;
         __syncwarp();  // every lane has read the centroids before they change
 #pragma unroll 1
         for (int j = 0; j < 16; ++j) {
@@ -219,6 +244,8 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
     const float loss = row_pairwise<W>(block_pairwise<M>(e2));
     if (!active)
         return;
+    if (a.row_iters && sub == 0)
+        a.row_iters[row] = it;
     uint8_t *cr = a.codes + row * a.codes_ld + kbase / 2;
 #pragma unroll
     for (int m = 0; m < (M + 1) / 2; ++m) {

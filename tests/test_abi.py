@@ -182,13 +182,13 @@ def test_embbag_bwd_no_entries_is_a_noop_and_workspace_size(L):
 
 
 @pytest.mark.parametrize("args,msg", [
-    ((NULL, -1, 16, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "n_rows"),
-    ((NULL, 4, 0, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "d = 0"),
-    ((NULL, 4, 16, 15, NULL, 8, NULL, NULL, 10, NULL, NULL), "x_ld"),
-    ((NULL, 4, 16, 16, NULL, 7, NULL, NULL, 10, NULL, NULL), "codes_ld"),
-    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, 65, NULL, NULL), "iters"),
-    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, -1, NULL, NULL), "iters"),
-    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, 10, NULL, NULL), "non-NULL"),
+    ((NULL, -1, 16, 16, NULL, 8, NULL, NULL, NULL, 10, NULL, NULL), "n_rows"),
+    ((NULL, 4, 0, 16, NULL, 8, NULL, NULL, NULL, 10, NULL, NULL), "d = 0"),
+    ((NULL, 4, 16, 15, NULL, 8, NULL, NULL, NULL, 10, NULL, NULL), "x_ld"),
+    ((NULL, 4, 16, 16, NULL, 7, NULL, NULL, NULL, 10, NULL, NULL), "codes_ld"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, NULL, 65, NULL, NULL), "iters"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, NULL, -1, NULL, NULL), "iters"),
+    ((NULL, 4, 16, 16, NULL, 8, NULL, NULL, NULL, 10, NULL, NULL), "non-NULL"),
 ])
 def test_kmeans_quantize_rejects(L, args, msg):
     assert L.dq_quantize_rows_kmeans4(*args) == dq.DQ_ERR_INVALID_ARG

@@ -69,6 +69,37 @@ def test_kmeans_iterations_and_values(cuda_device, iters, kind):
     _assert_same(_rows(1500, 64, iters + 7, kind), iters)
 
 
+@pytest.mark.parametrize("d,kind", [(16, "normal"), (64, "heavy"), (128, "offset"), (48, "few"), (1024, "normal")])
+def test_kmeans_stops_at_a_fixed_point(cuda_device, d, kind):
+    # the kernel stops a row once its assignment repeats; row_iters says after how many
+    # centroid updates. The oracle run for exactly that many iterations must give the
+    # outputs of all 64, and so must the GPU (with or without the counts requested).
+    n, iters = (257 if d == 1024 else 1200), 64
+    x = _rows(n, d, d + 11, kind)
+    xd = to_dev(x)
+    cld = (d + 1) // 2
+    got = []
+    for want_iters in (True, False):
+        codes = torch.zeros((n, cld), dtype=torch.uint8, device="cuda")
+        cb = torch.zeros((n, 16), dtype=torch.int16, device="cuda")
+        loss = torch.zeros(n, dtype=torch.float32, device="cuda")
+        its = torch.full((n,), -1, dtype=torch.int32, device="cuda") if want_iters else None
+        dq.dq_quantize_rows_kmeans4(xd, n, d, d, codes, cld, cb, loss, iters, None, None, row_iters=its)
+        got.append((codes.cpu().numpy(), cb.cpu().numpy().view(np.uint16), loss.cpu().numpy().view(np.uint32),
+                    its.cpu().numpy() if want_iters else None))
+    (gc, gcb, gl, it), (gc2, gcb2, gl2, _) = got
+    assert np.array_equal(gc, gc2) and np.array_equal(gcb, gcb2) and np.array_equal(gl, gl2)
+    oc, ocb, ol = oracle.quantize_rows_kmeans(x, iters=iters)
+    assert np.array_equal(gc, oc) and np.array_equal(gcb, ocb) and np.array_equal(gl, ol.view(np.uint32))
+    assert it.min() >= 0 and it.max() <= iters
+    assert it.mean() < iters / 2, it.mean()   # Lloyd's iteration settles long before 64 updates
+    for k in np.unique(it):
+        rows = np.nonzero(it == k)[0]
+        kc, kcb, kl = oracle.quantize_rows_kmeans(x[rows], iters=int(k))
+        assert np.array_equal(kc, oc[rows]) and np.array_equal(kcb, ocb[rows]), k
+        assert np.array_equal(kl.view(np.uint32), ol.view(np.uint32)[rows]), k
+
+
 def test_kmeans_special_rows_and_strides(cuda_device):
     x = _rows(600, 16, 3)
     x[0] = 0.0
