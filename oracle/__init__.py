@@ -72,6 +72,8 @@ def lib():
             L.oracle_quantize_rows_kmeans.restype = i32
             L.oracle_dequantize_rows_kmeans.argtypes = [vp, i64, vp, i64, i32, vp, i64]
             L.oracle_dequantize_rows_kmeans.restype = i32
+            L.oracle_kmeans_means.argtypes = [vp, vp, i32, vp]
+            L.oracle_kmeans_means.restype = i32
             L.oracle_embbag.restype = i64
             _lib = L
     return _lib
@@ -212,6 +214,19 @@ def quantize_rows_kmeans(x: np.ndarray, iters: int = KMEANS_ITERS, nthreads: int
     if rc != 0:
         raise ValueError("oracle_quantize_rows_kmeans: bad arguments")
     return codes, cb, loss
+
+
+def kmeans_means(x: np.ndarray, a: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """One centroid update of the codebook quantizer: the new c[16] from the row x and
+    its assignment a (clusters without members keep their c)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    a = np.ascontiguousarray(a, dtype=np.int32)
+    out = np.array(c, dtype=np.float32, copy=True)
+    if x.ndim != 1 or a.shape != x.shape or out.shape != (16,):
+        raise ValueError("kmeans_means: x and a of one row, c of 16")
+    if lib().oracle_kmeans_means(_p(x), _p(a), x.size, _p(out)) != 0:
+        raise ValueError("oracle_kmeans_means: bad arguments")
+    return out
 
 
 def dequantize_rows_kmeans(codes: np.ndarray, codebook: np.ndarray, d: int) -> np.ndarray:

@@ -66,16 +66,19 @@
  *   e. Each touched row (one with at least one entry) is quantized again from its new
  *      master values by the quantizer above (greedy or min/max); other rows keep
  *      their codes.
- * *   Codebook quantizer ("Post-Training 4-bit Quantization on Embedding Tables",
+ *   Codebook quantizer ("Post-Training 4-bit Quantization on Embedding Tables",
  *   提出的方法 bullet 3: codebook quantization by k-means, values mapped to a
  *   non-uniform set; 主要发现 bullet 3: the 18.8%-37.5% sizes fit 16 binary16 centroids
  *   per row). The pages fix no initialisation, iteration count or precision; the
  *   reading taken is one-dimensional Lloyd iterations in binary32:
  *   K1. c_j = fma(j, fl(R / 15), xmin), j = 0..15 (the min/max quantizer's levels).
  *   K2. `iters` times: a_k = the j minimising fl(|fl(x_k - c_j)|), ties to the lower j;
- *       then for every j with n_j > 0 members, c_j = fl(S_j / n_j) with S_j the pairwise
- *       sum (as the loss above) of x_k over the members (non-members add +0); an empty
- *       cluster keeps its centroid.
+ *       then for every j with n_j > 0 members, c_j = the mean of its members: their
+ *       values summed in binary64 from +0 in index order (one addition after the
+ *       other), divided by n_j in binary64, the quotient rounded once to binary32; an
+ *       empty cluster keeps its centroid. (The pages name the mean and no order; this
+ *       is the plainest order, and where every partial sum is exact in binary64, as
+ *       for most rows, the sum is the exact one and no order can change it.)
  *   K3. Stored centroids C_j = h(c_j); codes q_k = the j minimising fl(|fl(x_k - w(C_j))|),
  *       ties to the lower j; packed as above. Row loss: the pairwise sum of
  *       fl(fl(x_k - w(C_{q_k}))^2).
@@ -353,6 +356,35 @@ static int nearest(float x, const float *c)
     return best;
 }
 
+/* K2's update of the centroids c[16] from the assignment a[0..d-1]. */
+static void kmeans_means(const float *x, const int32_t *a, int d, float *c)
+{
+    double s[16];
+    int n[16];
+    for (int j = 0; j < 16; j++) {
+        s[j] = 0.0;
+        n[j] = 0;
+    }
+    for (int k = 0; k < d; k++) {
+        s[a[k]] += (double)x[k];
+        n[a[k]] += 1;
+    }
+    for (int j = 0; j < 16; j++)
+        if (n[j] > 0)
+            c[j] = (float)(s[j] / (double)n[j]);
+}
+
+int32_t oracle_kmeans_means(const float *x, const int32_t *a, int32_t d, float *c)
+{
+    if (d < 1 || d > ORACLE_MAX_D)
+        return -1;
+    for (int k = 0; k < d; k++)
+        if (a[k] < 0 || a[k] > 15)
+            return -1;
+    kmeans_means(x, a, d, c);
+    return 0;
+}
+
 /* Steps K1-K3 for one row; cbuf holds next_pow2(d) floats. Writes the stored
  * centroids (binary16), the packed codes, and returns the row loss. */
 static float kmeans_row(const float *x, int d, int iters, float *cbuf, uint8_t *codes, uint16_t *codebook)
@@ -367,20 +399,11 @@ static float kmeans_row(const float *x, int d, int iters, float *cbuf, uint8_t *
     for (int j = 0; j < 16; j++)
         c[j] = fmaf((float)j, step, xmin);
     int P = next_pow2(d);
-    int a[ORACLE_MAX_D];
+    int32_t a[ORACLE_MAX_D];
     for (int it = 0; it < iters; it++) {
         for (int k = 0; k < d; k++)
             a[k] = nearest(x[k], c);
-        for (int j = 0; j < 16; j++) {
-            int n = 0;
-            for (int k = 0; k < P; k++) {
-                int member = k < d && a[k] == j;
-                cbuf[k] = member ? x[k] : 0.0f;
-                n += member;
-            }
-            if (n > 0)
-                c[j] = pairwise_sum(cbuf, P) / (float)n;
-        }
+        kmeans_means(x, a, d, c);
     }
     float C[16];
     for (int j = 0; j < 16; j++) {

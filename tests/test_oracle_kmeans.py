@@ -4,9 +4,10 @@ section 提出的方法 (proposed method), bullet 3: codebook quantization by k-
 clustering; 主要发现 (main findings), bullet 3).
 
 Reading: centroids start at the 16 levels of the min/max quantizer; `iters` Lloyd
-iterations in binary32 (nearest centroid by |x - c|, ties to the lower index; mean by
-a pairwise sum over the members and one division; empty clusters keep their
-centroid); stored as binary16; final codes = nearest stored centroid."""
+iterations in binary32 (nearest centroid by |x - c|, ties to the lower index; the mean
+of a cluster = the binary64 sum of its members in index order / their count in
+binary64, rounded once to binary32; empty clusters keep their centroid); stored as
+binary16; final codes = nearest stored centroid."""
 from fractions import Fraction
 
 import numpy as np
@@ -138,3 +139,54 @@ def test_codebook_bag_sums_exactly():
         exact = [sum((Fraction(float(deq[i, k])) for i in idx[off[b]:off[b + 1]]), Fraction(0)) for k in range(d)]
         assert [float(v) for v in out[b]] == [float(round_to_f32(e)) for e in exact]
     assert skipped == 0
+
+
+def test_mean_sums_members_in_index_order():
+    # t = 2^-60 vanishes when added to 1 in binary64. Members [1, t, -1, t]: one addition
+    # after the other gives ((1 + t) - 1) + t = t, so the mean is t / 4 = 2^-62; a pairwise
+    # order would give (1 + t) + (-1 + t) = 0 and the exact mean is 2^-61
+    c0 = np.arange(16, dtype=np.float32)
+    a = np.full(4, 5, np.int32)
+    t = np.float32(2.0 ** -60)
+    got = oracle.kmeans_means(np.array([1.0, t, -1.0, t], np.float32), a, c0)
+    assert got[5] == np.float32(2.0 ** -62)
+    # [1, t, -1]: (1 + t) - 1 = 0, a +0 mean
+    got = oracle.kmeans_means(np.array([1.0, t, -1.0], np.float32), a[:3], c0)
+    assert got[5] == 0.0 and not np.signbit(got[5])
+    # the other clusters have no members and keep their centroids
+    assert np.array_equal(np.delete(got, 5), np.delete(c0, 5))
+
+
+def test_mean_of_exactly_summed_members_is_the_rounded_exact_mean():
+    # members on a 2^-20 grid below 2^10: every binary64 partial sum is exact, so the
+    # centroid is the exact mean rounded to binary32 -- once when the count is a power
+    # of two (the binary64 quotient is then exact too), and within binary32's half ulp
+    # plus binary64's quotient rounding otherwise
+    r = np.random.default_rng(7)
+    for trial in range(300):
+        d = int(r.integers(1, 200))
+        x = (r.integers(-2 ** 30, 2 ** 30, d) * 2.0 ** -20).astype(np.float32)
+        a = r.integers(0, 16, d).astype(np.int32)
+        c0 = r.standard_normal(16).astype(np.float32)
+        got = oracle.kmeans_means(x, a, c0)
+        for j in range(16):
+            m = a == j
+            n = int(m.sum())
+            if n == 0:
+                assert got[j] == c0[j]
+                continue
+            exact = sum((F(v) for v in x[m]), Fraction(0)) / n
+            want = round_to_f32(exact)
+            if n & (n - 1) == 0:
+                assert got[j] == want, (trial, j)
+            else:
+                assert abs(F(got[j]) - exact) <= abs(F(want) - exact) + abs(exact) * Fraction(1, 2 ** 52), (trial, j)
+
+
+def test_mean_step_keeps_empty_clusters_and_counts_every_member():
+    x = np.array([3.0, 5.0, -2.0, 7.0], np.float32)
+    a = np.array([2, 2, 9, 2], np.int32)
+    c0 = np.full(16, -1.0, np.float32)
+    got = oracle.kmeans_means(x, a, c0)
+    assert got[2] == np.float32(5.0) and got[9] == np.float32(-2.0)
+    assert np.all(np.delete(got, [2, 9]) == -1.0)
