@@ -210,8 +210,8 @@ dq_status dq_row_l2_error(const float *x, int64_t n_rows, int32_t d, int64_t x_l
  * The pages fix no algorithm details; this library computes, in binary32:
  *   1. c_j = fma(j, (xmax - xmin) / 15, xmin), j = 0..15.
  *   2. `iters` times: q_k = the j minimising |x_k - c_j| (ties to the lower j); for each
- *      j with members, c_j = (pairwise sum of its members, padded with +0 as the loss
- *      above) / (their count); a cluster without members keeps c_j.
+ *      j with members, c_j = their binary64 sum from +0 in index order / their count, the
+ *      binary64 quotient rounded to binary32; a cluster without members keeps c_j.
  *   3. codebook_j = fp16(c_j); codes = the nearest stored centroid (ties to the lower j);
  *      row_loss = pairwise sum of (x_k - codebook[q_k])^2.
  */

@@ -12,13 +12,16 @@
 // binary16 storage, final codes against the stored centroids.
 //
 // Layout as the greedy quantizer's: a row of d <= P = next_pow2(d) elements in
-// registers, W lanes per row, M = P / W contiguous elements per lane. A cluster's
-// member sum is the pairwise (recursive-halving) sum over the padded row: each lane
-// builds the tree of its aligned block bottom-up, and an XOR butterfly over the W
-// lanes joins the blocks in tree order; IEEE addition is commutative, so every lane
-// of a row ends with the identical sums and centroids. ALU bound: each iteration
-// costs 16 distance evaluations and 16 masked adds per element. A warp stops iterating
-// once every row's assignment has repeated (a fixed point of the iteration).
+// registers, W lanes per row, M = P / W contiguous elements per lane. A cluster's mean
+// is its members' binary64 sum in index order over their count. When the row's
+// nonzero values span at most 29 - ceil(log2 d) binades, every partial sum of its
+// members is an integer multiple of the smallest value's ulp below 2^53 of them, i.e.
+// exact in binary64, and any order gives the index-order sum: each element is then
+// added once into its own cluster's binary64 accumulator (one per lane, in shared
+// memory), and the W lanes' accumulators are added per cluster. Other rows (rare:
+// values near zero beside large ones, non-finite values) are summed by one lane per
+// row in index order. A warp stops iterating once every row's assignment has repeated
+// (a fixed point of the iteration).
 #include <cfloat>
 
 #include "dq_internal.cuh"
@@ -50,14 +53,20 @@ __device__ __forceinline__ float row_pairwise(float lane_sum)
     return lane_sum;
 }
 
-template <int W>
-__device__ __forceinline__ int row_count(int c)
-{
-#pragma unroll
-    for (int o = 1; o < W; o <<= 1)
-        c += __shfl_xor_sync(0xffffffffu, c, o);
-    return c;
-}
+// A warp's shared memory for the centroid update: per lane and cluster a binary64 sum
+// and a count ([cluster][lane]: the warp's accesses are conflict-free whatever the
+// clusters), or, on the sequential path, the lanes' elements and codes in index order.
+// One per warp, as warps of a block may take different paths.
+union KmeansUpdate {
+    struct {
+        double s[16][32];
+        int32_t n[16][32];
+    } acc;
+    struct {
+        float x[32 * 32];
+        uint8_t q[32 * 32];
+    } seq;
+};
 
 // q[m] = argmin_j fl(|fl(x[m] - c_j)|), ties to the lower j, for the lane's M elements;
 // the centroids are read from shared memory, one j at a time (a short loop body keeps
@@ -158,11 +167,34 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
             nonfinite |= !isfinite(x[m]);
         }
     }
+    // binary exponent fields of the lane's nonzero values (subnormals count as 1: the
+    // same ulp), for the row's span
+    int emax = 0, emin = 255;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const uint32_t u = __float_as_uint(x[m]) & 0x7fffffffu;
+        if ((FULL || kbase + m < d) && u != 0u) {
+            const int e = max((int)(u >> 23), 1);
+            emax = max(emax, e);
+            emin = min(emin, e);
+        }
+    }
+    int nf = nonfinite ? 1 : 0;
 #pragma unroll
     for (int o = 1; o < W; o <<= 1) {
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        emax = max(emax, __shfl_xor_sync(0xffffffffu, emax, o));
+        emin = min(emin, __shfl_xor_sync(0xffffffffu, emin, o));
+        nf |= __shfl_xor_sync(0xffffffffu, nf, o);
     }
+    const int clog2d = d > 1 ? 32 - __clz(d - 1) : 0;
+    const bool exact_row = nf == 0 && (emax == 0 || emax - emin <= 29 - clog2d);
+    const bool exact = __all_sync(0xffffffffu, exact_row);  // the warp's update path
+    __shared__ KmeansUpdate upd_all[4];
+    KmeansUpdate &upd = upd_all[threadIdx.x >> 5];
+    const int lane = threadIdx.x & 31;
+    const int row0 = lane & ~(W - 1);  // the row's first lane in the warp
     // the row's 16 centroids live in shared memory (every lane of the row writes the
     // same values; __syncwarp orders the writes before the reads)
     __shared__ float cs_all[128 / W][17];  // padded: rows' slots start in different banks
@@ -204,22 +236,62 @@ __global__ void __launch_bounds__(128) kmeans_rows_kernel(const KmeansArgs a)
         if (__all_sync(0xffffffffu, same))
             break;
         __syncwarp();  // every lane has read the centroids before they change
-#pragma unroll 1
-        for (int j = 0; j < 16; ++j) {
-            float v[M];
-            int cnt = 0;
+        if (exact) {
+            // every element into its own cluster's accumulator of this lane
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                upd.acc.s[j][lane] = 0.0;
+                upd.acc.n[j][lane] = 0;
+            }
 #pragma unroll
             for (int m = 0; m < M; ++m) {
-                const bool member = (FULL || kbase + m < d) && q[m] == j;
-                v[m] = member ? x[m] : 0.0f;
-                cnt += member;
+                if (FULL || kbase + m < d) {
+                    const int j = q[m];
+                    upd.acc.s[j][lane] += (double)x[m];
+                    upd.acc.n[j][lane] += 1;
+                }
             }
-            const float sj = row_pairwise<W>(block_pairwise<M>(v));
-            const int nj = row_count<W>(cnt);
-            if (sub == 0 && nj > 0)
-                c[j] = __fdiv_rn(sj, (float)nj);
+            __syncwarp();
+            // lane `sub` of the row takes clusters sub, sub + W, ...
+            for (int j = sub; j < 16; j += W) {
+                double sj = 0.0;
+                int nj = 0;
+#pragma unroll 4
+                for (int l = 0; l < W; ++l) {
+                    sj += upd.acc.s[j][row0 + l];
+                    nj += upd.acc.n[j][row0 + l];
+                }
+                if (nj > 0)
+                    c[j] = __double2float_rn(__ddiv_rn(sj, (double)nj));
+            }
+        } else {
+            // one lane per row adds the members in index order
+#pragma unroll
+            for (int m = 0; m < M; ++m) {
+                upd.seq.x[lane * M + m] = x[m];
+                upd.seq.q[lane * M + m] = q[m];
+            }
+            __syncwarp();
+            if (sub == 0) {
+                double sj[16];
+                int nj[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    sj[j] = 0.0;
+                    nj[j] = 0;
+                }
+                for (int k = 0; k < d; ++k) {
+                    const int j = upd.seq.q[row0 * M + k];
+                    sj[j] += (double)upd.seq.x[row0 * M + k];
+                    nj[j] += 1;
+                }
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (nj[j] > 0)
+                        c[j] = __double2float_rn(__ddiv_rn(sj[j], (double)nj[j]));
+            }
         }
-        __syncwarp();
+        __syncwarp();  // the updated centroids, and the accumulators free again
     }
     // K3: binary16 centroids, final codes, loss
     __half h[16];

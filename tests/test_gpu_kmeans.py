@@ -100,6 +100,26 @@ def test_kmeans_stops_at_a_fixed_point(cuda_device, d, kind):
         assert np.array_equal(kl.view(np.uint32), ol.view(np.uint32)[rows]), k
 
 
+@pytest.mark.parametrize("d", [3, 16, 64, 128, 1024])
+def test_kmeans_exact_and_sequential_updates(cuda_device, d):
+    # a row whose nonzero values span more binades than binary64 sums hold exactly is
+    # updated in index order by one lane; the others add each element into its own
+    # cluster in any order. Rows of both kinds share warps and blocks here.
+    r = np.random.default_rng(d + 40)
+    n = 300 if d == 1024 else 3000
+    x = r.standard_normal((n, d)).astype(np.float32)
+    wide = r.random(n) < 0.1
+    for i in np.nonzero(wide)[0]:
+        k = r.integers(0, d, 3 if d > 3 else 1)
+        x[i, k] = np.float32(r.choice([1e-12, -3e-15, 2e-39, 1e-30]))
+    # cancellation inside a cluster: values around 0 at scales 2^-40 apart
+    for i in np.nonzero(r.random(n) < 0.05)[0]:
+        k = r.integers(0, d, 4 if d >= 4 else d)
+        x[i, k] = np.float32([1e-3, 1e-3 * 2.0 ** -40, -1e-3, 1e-3 * 2.0 ** -41])[:k.size]
+    _assert_same(x, 10)
+    _assert_same(x, 64)
+
+
 def test_kmeans_special_rows_and_strides(cuda_device):
     x = _rows(600, 16, 3)
     x[0] = 0.0
