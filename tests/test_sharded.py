@@ -175,6 +175,20 @@ def test_sharded_rejects_bad_shapes():
         with pytest.raises(ValueError, match="owner ranks"):
             sharded_embbag(tables, [0, 1, 0], D, torch.from_numpy(idx), torch.from_numpy(off), 4,
                            lookup=_oracle_lookup)
+        # the direct form checks its buffers, tables and offsets before any barrier or launch
+        from int4_row_wise_b200.sharded import OwnerBuffers, sharded_embbag_direct
+        ti, to = torch.from_numpy(idx), torch.from_numpy(off)
+        good = OwnerBuffers(torch.zeros((4, 3 * D)), [0], [])
+        with pytest.raises(ValueError, match="owner buffers"):
+            sharded_embbag_direct(tables, owner, D, ti, to, 4, OwnerBuffers(good.own, [0, 0], []))
+        with pytest.raises(ValueError, match="own buffer"):
+            sharded_embbag_direct(tables, owner, D, ti, to, 4, OwnerBuffers(torch.zeros((4, 2 * D)), [0], []))
+        with pytest.raises(ValueError, match="owns 3 tables"):
+            sharded_embbag_direct(tables[:2], owner, D, ti, to, 4, good)
+        with pytest.raises(ValueError, match="offsets"):
+            sharded_embbag_direct(tables, owner, D, ti, to[:-1], 4, good)
+        with pytest.raises(ValueError, match="owner ranks"):
+            sharded_embbag_direct(tables, [0, 1, 0], D, ti, to, 4, good)
     finally:
         dist.destroy_process_group()
 
