@@ -239,11 +239,20 @@ class OracleBench:
                 f"dequantized ({r['dequantize_s']:.3f} s), plus one full lookup call over {self.tables_kind} "
                 f"({r['lookup_s']:.3f} s)")
 
+    def single_core(self, n: int = 10_000) -> dict:
+        """The oracle quantizer alone on one thread, over the first n rows of the largest table."""
+        x = self.pool[int(np.argmax(self.wl.rows))][:n]
+        t0 = time.perf_counter()
+        self.oracle.quantize_rows(x, nthreads=1)
+        dt = time.perf_counter() - t0
+        return {"value": x.shape[0] / dt, "unit": "rows/s", "cores": 1, "rows": int(x.shape[0]),
+                "what": "the oracle's greedy quantizer on one thread, first rows of the largest table"}
+
     def baseline(self, target_s: float) -> dict:
         r = self.step(target_s)
         return {"value": r["rows"] / r["step_s"], "unit": "rows/s", "cores": self.cores, "kind": "oracle",
                 "sample": self.describe(r), "timed_s": r["step_s"],
-                "extrapolated_full_step_s": r["full_step_s"]}
+                "extrapolated_full_step_s": r["full_step_s"], "single_core": self.single_core()}
 
 
 def run_reference(args, wl: W.Workload) -> None:
