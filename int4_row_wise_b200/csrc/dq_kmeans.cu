@@ -374,21 +374,36 @@ __global__ void __launch_bounds__(256) kmeans_dequant_kernel(const KmeansDequant
     }
 }
 
-// One warp per bag (t, b); lane l owns elements l, l + 32, ...; per id, lanes 0..15 read
-// the row's 16 centroids and each lane takes its element's centroid by shuffle. The
-// sum runs in binary32 in id order, so a bag of one id returns the dequantized row.
+// One warp per bag (t, b); lane l owns elements l, l + 32, ... (CH chunks of 32); per id,
+// lanes 0..15 read the row's 16 centroids and each lane takes its elements' centroids by
+// shuffle. The sum runs in binary32 in id order, so a bag of one id returns the
+// dequantized row. The next bag's offsets, and the id at its own position (where a
+// one-id bag of an all-one-hot call keeps it), are loaded while the current bag is summed.
+template <int CH>
 __global__ void __launch_bounds__(256) kmeans_bag_kernel(const KmeansBagTables tabs, const KmeansBagArgs a)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t G = (int64_t)a.T * a.batch;
-    const int32_t total = a.offsets[G];
-    const int chunks = (a.d + 31) / 32;
+    const int32_t total = __ldg(a.offsets + G);
+    int32_t np0 = 0, np1 = 0, nid = -1;
+    if (warp < G) {
+        np0 = __ldg(a.offsets + warp);
+        np1 = __ldg(a.offsets + warp + 1);
+        nid = warp < total ? __ldg(a.indices + warp) : -1;
+    }
     for (int64_t g = warp; g < G; g += warps) {
+        int32_t p0 = np0, p1 = np1;
+        const int32_t own = nid;
+        const int64_t gn = g + warps;
+        if (gn < G) {
+            np0 = __ldg(a.offsets + gn);
+            np1 = __ldg(a.offsets + gn + 1);
+            nid = gn < total ? __ldg(a.indices + gn) : -1;
+        }
         const int t = (int)div_batch((uint32_t)g, a.div);
         const int64_t b = g - (int64_t)t * a.batch;
-        int32_t p0 = a.offsets[g], p1 = a.offsets[g + 1];
         p0 = p0 < 0 ? 0 : (p0 > total ? total : p0);
         p1 = p1 < 0 ? 0 : (p1 > total ? total : p1);
         if (p1 < p0) {
@@ -397,27 +412,37 @@ __global__ void __launch_bounds__(256) kmeans_bag_kernel(const KmeansBagTables t
             p1 = p0;
         }
         const int64_t n_rows = tabs.n_rows[t];
-        float *out = a.out + b * (int64_t)a.T * a.d + (int64_t)t * a.d;
-        for (int ch = 0; ch < chunks; ++ch) {
-            const int k = ch * 32 + lane;
-            float acc = 0.0f;
-            for (int32_t p = p0; p < p1; ++p) {
-                const int32_t id = __ldg(a.indices + p);
-                if (id < 0 || id >= n_rows) {
-                    if (lane == 0 && ch == 0)
-                        raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
-                    continue;
-                }
-                const float cj = lane < 16 ? __half2float(__ushort_as_half(__ldg(tabs.codebook[t] + 16 * (int64_t)id + lane)))
-                                           : 0.0f;
+        const uint16_t *cbt = tabs.codebook[t];
+        const uint8_t *ct = tabs.codes[t];
+        const int64_t cld = tabs.codes_ld[t];
+        float acc[CH];
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch)
+            acc[ch] = 0.0f;
+        for (int32_t p = p0; p < p1; ++p) {
+            const int32_t id = (int64_t)p == g ? own : __ldg(a.indices + p);
+            if (id < 0 || id >= n_rows) {
+                if (lane == 0)
+                    raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                continue;
+            }
+            const float cj = lane < 16 ? __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id + lane))) : 0.0f;
+            const uint8_t *cr = ct + (int64_t)id * cld;
+#pragma unroll
+            for (int ch = 0; ch < CH; ++ch) {
+                const int k = ch * 32 + lane;
                 unsigned qk = 0;
                 if (k < a.d)
-                    qk = (__ldg(tabs.codes[t] + (int64_t)id * tabs.codes_ld[t] + k / 2) >> (4 * (k & 1))) & 15u;
-                const float v = __shfl_sync(0xffffffffu, cj, (int)qk);
-                acc = __fadd_rn(acc, v);
+                    qk = (__ldg(cr + k / 2) >> (4 * (k & 1))) & 15u;
+                acc[ch] = __fadd_rn(acc[ch], __shfl_sync(0xffffffffu, cj, (int)qk));
             }
+        }
+        float *out = a.out + b * (int64_t)a.T * a.d + (int64_t)t * a.d;
+#pragma unroll
+        for (int ch = 0; ch < CH; ++ch) {
+            const int k = ch * 32 + lane;
             if (k < a.d)
-                out[k] = acc;
+                out[k] = acc[ch];
         }
     }
 }
@@ -459,7 +484,20 @@ cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &
     const int64_t G = (int64_t)a.T * a.batch;
     const int64_t need = (G * 32 + 255) / 256;
     const int64_t cap = (int64_t)num_sms * 16;
-    kmeans_bag_kernel<<<(unsigned)(need < cap ? need : cap), 256, 0, stream>>>(tabs, a);
+    const unsigned grid = (unsigned)(need < cap ? need : cap);
+    const int chunks = (a.d + 31) / 32;
+    if (chunks <= 1)
+        kmeans_bag_kernel<1><<<grid, 256, 0, stream>>>(tabs, a);
+    else if (chunks <= 2)
+        kmeans_bag_kernel<2><<<grid, 256, 0, stream>>>(tabs, a);
+    else if (chunks <= 4)
+        kmeans_bag_kernel<4><<<grid, 256, 0, stream>>>(tabs, a);
+    else if (chunks <= 8)
+        kmeans_bag_kernel<8><<<grid, 256, 0, stream>>>(tabs, a);
+    else if (chunks <= 16)
+        kmeans_bag_kernel<16><<<grid, 256, 0, stream>>>(tabs, a);
+    else
+        kmeans_bag_kernel<32><<<grid, 256, 0, stream>>>(tabs, a);
     return cudaGetLastError();
 }
 
