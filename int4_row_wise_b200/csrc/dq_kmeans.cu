@@ -380,13 +380,12 @@ __global__ void __launch_bounds__(256) kmeans_dequant_kernel(const KmeansDequant
 // dequantized row. The next bag's offsets, and the id at its own position (where a
 // one-id bag of an all-one-hot call keeps it), are loaded while the current bag is summed.
 template <int CH>
-__global__ void __launch_bounds__(256) kmeans_bag_kernel(const KmeansBagTables tabs, const KmeansBagArgs a)
+__device__ __forceinline__ void bag_per_warp(const KmeansBagTables &tabs, const KmeansBagArgs &a, int64_t G,
+                                             int32_t total)
 {
     const int lane = threadIdx.x & 31;
     const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t G = (int64_t)a.T * a.batch;
-    const int32_t total = __ldg(a.offsets + G);
     int32_t np0 = 0, np1 = 0, nid = -1;
     if (warp < G) {
         np0 = __ldg(a.offsets + warp);
@@ -447,6 +446,166 @@ __global__ void __launch_bounds__(256) kmeans_bag_kernel(const KmeansBagTables t
     }
 }
 
+// Short bags (under two ids on average): a warp takes 32 consecutive bags. Lane j does bag
+// j's bookkeeping (offsets, the id, row pointers, output row) into a per-warp table in
+// shared memory; then the warp writes the bags' rows in groups of 8, with the 8 bags'
+// centroids and codes loaded before any is decoded (lanes 0..15 hold a centroid each,
+// every lane CH code bytes). Empty bags and bags of an invalid id write +0; bags of two or
+// more ids are summed afterwards, one at a time, in id order.
+constexpr int64_t kTileMinBags = 65536;   // 2048 tiles of 32 bags: enough to fill the GPU
+
+struct CbSlot {
+    const uint16_t *cb;   // the row's 16 centroids (one-id bags)
+    const uint8_t *cr;    // the row's codes
+    float *out;           // the bag's output row
+    int32_t p0, p1;       // the clamped offsets (bags of two or more ids)
+    int32_t kind;         // 0: one valid id, 1: write +0, 2: two or more ids
+    int32_t t;
+};
+
+template <int CH>
+__device__ __forceinline__ void bag_tiles(const KmeansBagTables &tabs, const KmeansBagArgs &a, int64_t G,
+                                          int32_t total, CbSlot *slots)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t wpb = blockDim.x >> 5;
+    for (int64_t g0 = ((int64_t)blockIdx.x * wpb + (threadIdx.x >> 5)) * 32; g0 < G; g0 += (int64_t)gridDim.x * wpb * 32) {
+        const int64_t g = g0 + lane;
+        unsigned multi = 0;
+        if (g < G) {
+            int32_t p0 = __ldg(a.offsets + g), p1 = __ldg(a.offsets + g + 1);
+            const int32_t own = g < total ? __ldg(a.indices + g) : -1;
+            p0 = p0 < 0 ? 0 : (p0 > total ? total : p0);
+            p1 = p1 < 0 ? 0 : (p1 > total ? total : p1);
+            if (p1 < p0) {
+                raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
+                p1 = p0;
+            }
+            const int t = (int)div_batch((uint32_t)g, a.div);
+            const int64_t b = g - (int64_t)t * a.batch;
+            CbSlot sl;
+            sl.out = a.out + b * (int64_t)a.T * a.d + (int64_t)t * a.d;
+            sl.p0 = p0;
+            sl.p1 = p1;
+            sl.t = t;
+            sl.cb = nullptr;
+            sl.cr = nullptr;
+            sl.kind = 1;
+            if (p1 == p0 + 1) {
+                const int32_t id = (int64_t)p0 == g ? own : __ldg(a.indices + p0);
+                if (id >= 0 && (int64_t)id < tabs.n_rows[t]) {
+                    sl.cb = tabs.codebook[t] + 16 * (int64_t)id;
+                    sl.cr = tabs.codes[t] + (int64_t)id * tabs.codes_ld[t];
+                    sl.kind = 0;
+                } else {
+                    raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                }
+            } else if (p1 > p0 + 1) {
+                sl.kind = 2;
+            }
+            slots[lane] = sl;
+        }
+        multi = __ballot_sync(0xffffffffu, g < G && slots[lane].kind == 2);
+        __syncwarp();
+        const int nb = (int)min((int64_t)32, G - g0);
+        for (int j0 = 0; j0 < nb; j0 += 8) {
+            float cj[8];
+            unsigned q[8][CH];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u;
+                const bool one = j < nb && slots[j].kind == 0;
+                cj[u] = (one && lane < 16) ? __half2float(__ushort_as_half(__ldg(slots[j].cb + lane))) : 0.0f;
+#pragma unroll
+                for (int ch = 0; ch < CH; ++ch) {
+                    const int k = ch * 32 + lane;
+                    q[u][ch] = (one && k < a.d) ? (unsigned)__ldg(slots[j].cr + k / 2) : 0u;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = j0 + u;
+                if (j >= nb)
+                    break;
+                const int kind = slots[j].kind;   // warp-uniform
+                if (kind == 2)
+                    continue;
+                float *o = slots[j].out;
+#pragma unroll
+                for (int ch = 0; ch < CH; ++ch) {
+                    const int k = ch * 32 + lane;
+                    const unsigned qk = (q[u][ch] >> (4 * (k & 1))) & 15u;
+                    const float v = __shfl_sync(0xffffffffu, cj[u], (int)qk);
+                    if (k < a.d)
+                        o[k] = kind == 0 ? __fadd_rn(0.0f, v) : 0.0f;
+                }
+            }
+        }
+        while (multi) {   // bags of two or more ids, one at a time
+            const int j = __ffs(multi) - 1;
+            multi &= multi - 1;
+            const CbSlot sl = slots[j];
+            const int64_t n_rows = tabs.n_rows[sl.t];
+            const uint16_t *cbt = tabs.codebook[sl.t];
+            const uint8_t *ct = tabs.codes[sl.t];
+            const int64_t cld = tabs.codes_ld[sl.t];
+            float acc[CH];
+#pragma unroll
+            for (int ch = 0; ch < CH; ++ch)
+                acc[ch] = 0.0f;
+            for (int32_t p = sl.p0; p < sl.p1; ++p) {
+                const int32_t id = __ldg(a.indices + p);
+                if (id < 0 || id >= n_rows) {
+                    if (lane == 0)
+                        raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                    continue;
+                }
+                const float c = lane < 16 ? __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id + lane))) : 0.0f;
+                const uint8_t *cr = ct + (int64_t)id * cld;
+#pragma unroll
+                for (int ch = 0; ch < CH; ++ch) {
+                    const int k = ch * 32 + lane;
+                    unsigned qk = 0;
+                    if (k < a.d)
+                        qk = (__ldg(cr + k / 2) >> (4 * (k & 1))) & 15u;
+                    acc[ch] = __fadd_rn(acc[ch], __shfl_sync(0xffffffffu, c, (int)qk));
+                }
+            }
+#pragma unroll
+            for (int ch = 0; ch < CH; ++ch) {
+                const int k = ch * 32 + lane;
+                if (k < a.d)
+                    sl.out[k] = acc[ch];
+            }
+        }
+        __syncwarp();   // the slots are rewritten by the next tile
+    }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(256) kmeans_bag_kernel(const __grid_constant__ KmeansBagTables tabs,
+                                                         const KmeansBagArgs a)
+{
+    const int64_t G = (int64_t)a.T * a.batch;
+    bag_per_warp<CH>(tabs, a, G, __ldg(a.offsets + G));
+}
+
+// Calls of many bags at d <= 64: the id count (the last offset) picks the layout, 32 bags
+// per warp when the bags hold under two ids on average, else one warp per bag. (A kernel
+// of its own: the tile layout's registers would cost the smaller calls occupancy.)
+template <int CH>
+__global__ void __launch_bounds__(256) kmeans_bag_tile_kernel(const __grid_constant__ KmeansBagTables tabs,
+                                                              const KmeansBagArgs a)
+{
+    __shared__ CbSlot slots_all[8][32];
+    const int64_t G = (int64_t)a.T * a.batch;
+    const int32_t total = __ldg(a.offsets + G);
+    if ((int64_t)total < 2 * G)
+        bag_tiles<CH>(tabs, a, G, total, slots_all[threadIdx.x >> 5]);
+    else
+        bag_per_warp<CH>(tabs, a, G, total);
+}
+
 } // namespace
 
 cudaError_t launch_kmeans(const KmeansArgs &a, cudaStream_t stream)
@@ -486,6 +645,13 @@ cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &
     const int64_t cap = (int64_t)num_sms * 16;
     const unsigned grid = (unsigned)(need < cap ? need : cap);
     const int chunks = (a.d + 31) / 32;
+    if (G >= kTileMinBags && chunks <= 2) {
+        if (chunks <= 1)
+            kmeans_bag_tile_kernel<1><<<grid, 256, 0, stream>>>(tabs, a);
+        else
+            kmeans_bag_tile_kernel<2><<<grid, 256, 0, stream>>>(tabs, a);
+        return cudaGetLastError();
+    }
     if (chunks <= 1)
         kmeans_bag_kernel<1><<<grid, 256, 0, stream>>>(tabs, a);
     else if (chunks <= 2)

@@ -182,7 +182,7 @@ def _kmeans_tables(rows, d, seed):
 
 
 @pytest.mark.parametrize("d,pool", [(16, (1, 1)), (16, (0, 10)), (64, (20, 80)), (128, (1, 1)), (37, (0, 5)),
-                                    (256, (3, 9)), (512, (0, 3)), (1024, (1, 1)), (1000, (1, 4))])
+                                    (256, (3, 9)), (512, (0, 3)), (1024, (1, 1)), (1000, (1, 4)), (64, (0, 2))])
 def test_kmeans_bag(cuda_device, d, pool):
     rows = [500, 0, 1300] if pool != (1, 1) else [800, 1200]
     T, B = len(rows), 300
@@ -199,4 +199,29 @@ def test_kmeans_bag(cuda_device, d, pool):
     bag_tolerance_check(got, want, mag)
     if pool == (1, 1):
         assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+    assert bool(fl.item() & dq.DQ_FLAG_BAD_INDEX) == (skipped > 0)
+
+
+@pytest.mark.parametrize("d,pool", [(16, (1, 1)), (64, (1, 1)), (64, (0, 2)), (33, (0, 3)), (48, (1, 2)),
+                                    (64, (2, 6)), (16, (3, 5))])
+def test_kmeans_bag_many_bags(cuda_device, d, pool):
+    # 81,000 bags at d <= 64: under two ids on average they take the 32-bags-per-warp layout
+    # (one lane per bag for the bookkeeping, eight bags' rows loaded together), otherwise one
+    # warp per bag; empty bags, invalid ids (the empty middle table) and bags of two or more
+    # ids mixed in
+    rows = [700, 0, 1500]
+    T, B = len(rows), 27000
+    tabs = _kmeans_tables(rows, d, d + 5)
+    r = np.random.default_rng(d * 7 + pool[1])
+    lens = r.integers(pool[0], pool[1] + 1, T * B)
+    off = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    idx = np.concatenate([r.integers(0, max(rows[g // B], 1), lens[g]) if rows[g // B] else np.full(lens[g], 3)
+                          for g in range(T * B)]).astype(np.int32)
+    fl = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dt = [dq.KmeansTable(to_dev(c), to_dev(cb.view(np.int16))) for c, cb in tabs]
+    got = dq.embbag_kmeans(dt, d, to_dev(idx), to_dev(off), B, d_flags=fl).cpu().numpy()
+    want, mag, skipped = oracle.embbag(tabs, d, idx, off, B, with_abs_sum=True, codebook=True)
+    bag_tolerance_check(got, want, mag)
+    one = np.repeat(np.diff(off.astype(np.int64)).reshape(T, B).T == 1, d, axis=1)
+    assert np.array_equal(got[one].view(np.uint32), want[one].view(np.uint32))
     assert bool(fl.item() & dq.DQ_FLAG_BAD_INDEX) == (skipped > 0)
