@@ -590,6 +590,104 @@ __global__ void __launch_bounds__(256) kmeans_bag_kernel(const __grid_constant__
     bag_per_warp<CH>(tabs, a, G, __ldg(a.offsets + G));
 }
 
+// Rows of d = 16·E elements with E/2-byte aligned code pieces: each half-warp takes every
+// other id of the bag, its 16 lanes holding the row's 16 centroids and each lane decoding E
+// consecutive elements from one E/2-byte load; the halves' sums are added at the end (two
+// interleaved id-order sums: a bag of one id still returns the dequantized row).
+template <int E>
+__device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t (&w)[(E + 7) / 8])
+{
+    if constexpr (E == 4)
+        w[0] = __ldg(reinterpret_cast<const uint16_t *>(p));
+    else if constexpr (E == 8)
+        w[0] = __ldg(reinterpret_cast<const uint32_t *>(p));
+    else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2 *>(p));
+        w[0] = v.x;
+        w[1] = v.y;
+    }
+}
+
+template <int E>
+__global__ void __launch_bounds__(256) kmeans_bag_half_kernel(const __grid_constant__ KmeansBagTables tabs,
+                                                              const KmeansBagArgs a)
+{
+    constexpr int NW = (E + 7) / 8;
+    const int lane = threadIdx.x & 31;
+    const int h = lane >> 4, c = lane & 15;
+    const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t G = (int64_t)a.T * a.batch;
+    const int32_t total = __ldg(a.offsets + G);
+    int32_t np0 = 0, np1 = 0, nid = -1;
+    if (warp < G) {
+        np0 = __ldg(a.offsets + warp);
+        np1 = __ldg(a.offsets + warp + 1);
+        nid = warp < total ? __ldg(a.indices + warp) : -1;
+    }
+    for (int64_t g = warp; g < G; g += warps) {
+        int32_t p0 = np0, p1 = np1;
+        const int32_t own = nid;
+        const int64_t gn = g + warps;
+        if (gn < G) {
+            np0 = __ldg(a.offsets + gn);
+            np1 = __ldg(a.offsets + gn + 1);
+            nid = gn < total ? __ldg(a.indices + gn) : -1;
+        }
+        const int t = (int)div_batch((uint32_t)g, a.div);
+        const int64_t b = g - (int64_t)t * a.batch;
+        p0 = p0 < 0 ? 0 : (p0 > total ? total : p0);
+        p1 = p1 < 0 ? 0 : (p1 > total ? total : p1);
+        if (p1 < p0) {
+            if (lane == 0)
+                raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
+            p1 = p0;
+        }
+        const int64_t n_rows = tabs.n_rows[t];
+        const uint16_t *cbt = tabs.codebook[t];
+        const uint8_t *ct = tabs.codes[t] + c * (E / 2);
+        const int64_t cld = tabs.codes_ld[t];
+        float acc[E];
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            acc[e] = 0.0f;
+        bool bad = false;
+        for (int32_t q0 = p0; q0 < p1; q0 += 2) {   // this half's id: q0 + h
+            const int32_t p = q0 + h;
+            int32_t id = -1;
+            if (p < p1)
+                id = (int64_t)p == g ? own : __ldg(a.indices + p);
+            const bool ok = id >= 0 && (int64_t)id < n_rows;
+            bad |= p < p1 && !ok;
+            float cj = 0.0f;
+            uint32_t w[NW];
+#pragma unroll
+            for (int k = 0; k < NW; ++k)
+                w[k] = 0u;
+            if (ok) {
+                cj = __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id + c)));
+                load_codes<E>(ct + (int64_t)id * cld, w);
+            }
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                const unsigned qk = (w[e / 8] >> (4 * (e % 8))) & 15u;
+                const float v = __shfl_sync(0xffffffffu, cj, (h << 4) | (int)qk);
+                if (ok)
+                    acc[e] = __fadd_rn(acc[e], v);
+            }
+        }
+        if (__any_sync(0xffffffffu, bad) && lane == 0)
+            raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+        float *out = a.out + b * (int64_t)a.T * a.d + (int64_t)t * a.d + c * E;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            const float other = __shfl_xor_sync(0xffffffffu, acc[e], 16);
+            if (h == 0)
+                out[e] = __fadd_rn(acc[e], other);
+        }
+    }
+}
+
 // Calls of many bags at d <= 64: the id count (the last offset) picks the layout, 32 bags
 // per warp when the bags hold under two ids on average, else one warp per bag. (A kernel
 // of its own: the tile layout's registers would cost the smaller calls occupancy.)
@@ -650,6 +748,20 @@ cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &
             kmeans_bag_tile_kernel<1><<<grid, 256, 0, stream>>>(tabs, a);
         else
             kmeans_bag_tile_kernel<2><<<grid, 256, 0, stream>>>(tabs, a);
+        return cudaGetLastError();
+    }
+    // d = 64, 128, 256 with every table's code rows E/2-byte aligned: two ids per warp
+    const int E = a.d / 16;
+    bool half = (a.d == 64 || a.d == 128 || a.d == 256);
+    for (int t = 0; half && t < a.T; ++t)
+        half = tabs.codes_ld[t] % (E / 2) == 0 && (reinterpret_cast<uintptr_t>(tabs.codes[t]) % (E / 2)) == 0;
+    if (half) {
+        if (E == 4)
+            kmeans_bag_half_kernel<4><<<grid, 256, 0, stream>>>(tabs, a);
+        else if (E == 8)
+            kmeans_bag_half_kernel<8><<<grid, 256, 0, stream>>>(tabs, a);
+        else
+            kmeans_bag_half_kernel<16><<<grid, 256, 0, stream>>>(tabs, a);
         return cudaGetLastError();
     }
     if (chunks <= 1)
