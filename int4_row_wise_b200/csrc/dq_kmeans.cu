@@ -591,9 +591,10 @@ __global__ void __launch_bounds__(256) kmeans_bag_kernel(const __grid_constant__
 }
 
 // Rows of d = 16·E elements with E/2-byte aligned code pieces: each half-warp takes every
-// other id of the bag, its 16 lanes holding the row's 16 centroids and each lane decoding E
-// consecutive elements from one E/2-byte load; the halves' sums are added at the end (two
-// interleaved id-order sums: a bag of one id still returns the dequantized row).
+// other id of the bag (two of them loaded before either is added), its 16 lanes holding the
+// row's 16 centroids and each lane decoding E consecutive elements from one E/2-byte load;
+// the halves' sums are added at the end (two interleaved id-order sums: a bag of one id still
+// returns the dequantized row).
 template <int E>
 __device__ __forceinline__ void load_codes(const uint8_t *p, uint32_t (&w)[(E + 7) / 8])
 {
@@ -652,28 +653,37 @@ __global__ void __launch_bounds__(256) kmeans_bag_half_kernel(const __grid_const
         for (int e = 0; e < E; ++e)
             acc[e] = 0.0f;
         bool bad = false;
-        for (int32_t q0 = p0; q0 < p1; q0 += 2) {   // this half's id: q0 + h
-            const int32_t p = q0 + h;
-            int32_t id = -1;
-            if (p < p1)
-                id = (int64_t)p == g ? own : __ldg(a.indices + p);
-            const bool ok = id >= 0 && (int64_t)id < n_rows;
-            bad |= p < p1 && !ok;
-            float cj = 0.0f;
-            uint32_t w[NW];
+        for (int32_t q0 = p0; q0 < p1; q0 += 4) {   // this half's ids: q0 + h, q0 + 2 + h
+            int32_t id[2];
+            bool ok[2];
+            float cj[2];
+            uint32_t w[2][NW];
 #pragma unroll
-            for (int k = 0; k < NW; ++k)
-                w[k] = 0u;
-            if (ok) {
-                cj = __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id + c)));
-                load_codes<E>(ct + (int64_t)id * cld, w);
+            for (int u = 0; u < 2; ++u) {
+                const int32_t p = q0 + 2 * u + h;
+                id[u] = -1;
+                if (p < p1)
+                    id[u] = (int64_t)p == g ? own : __ldg(a.indices + p);
+                ok[u] = id[u] >= 0 && (int64_t)id[u] < n_rows;
+                bad |= p < p1 && !ok[u];
+                cj[u] = 0.0f;
+#pragma unroll
+                for (int k = 0; k < NW; ++k)
+                    w[u][k] = 0u;
+                if (ok[u]) {
+                    cj[u] = __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id[u] + c)));
+                    load_codes<E>(ct + (int64_t)id[u] * cld, w[u]);
+                }
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                const unsigned qk = (w[e / 8] >> (4 * (e % 8))) & 15u;
-                const float v = __shfl_sync(0xffffffffu, cj, (h << 4) | (int)qk);
-                if (ok)
-                    acc[e] = __fadd_rn(acc[e], v);
+            for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const unsigned qk = (w[u][e / 8] >> (4 * (e % 8))) & 15u;
+                    const float v = __shfl_sync(0xffffffffu, cj[u], (h << 4) | (int)qk);
+                    if (ok[u])
+                        acc[e] = __fadd_rn(acc[e], v);
+                }
             }
         }
         if (__any_sync(0xffffffffu, bad) && lane == 0)
