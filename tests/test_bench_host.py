@@ -1,6 +1,7 @@
 """bench.py's host-side pieces on CPU: the pooled table generation matches the serial
-one, the oracle baseline reports what it timed, and the lookup's algorithmic bytes
-count each table's distinct rows once."""
+one, the oracle baseline reports what it timed, the lookup's algorithmic bytes count
+each table's distinct rows once, and the codebook quantizer's work counts the updates
+it ran."""
 import numpy as np
 
 import bench
@@ -34,3 +35,17 @@ def test_oracle_baseline_reports_the_timed_sample():
     rows = int(r["sample"].split()[0])
     assert abs(r["value"] - rows / r["timed_s"]) < 1e-9 * r["value"]
     assert r["extrapolated_full_step_s"] > r["timed_s"]
+    sc = r["single_core"]
+    assert sc["cores"] == 1 and 0 < sc["rows"] <= 10_000 and sc["value"] > 0
+
+
+def test_kmeans_ops_count_the_updates_run():
+    import torch
+    # per element: 33 ops per update run, 32 more for a row that stopped before `iters`
+    # (the assignment that found the repeat), 35 for the final assignment and loss
+    its = [torch.tensor([10, 3, 0], dtype=torch.int32), torch.tensor([2], dtype=torch.int32)]
+    ops, per_row = bench._kmeans_ops(64, 10, its)
+    assert ops == 64 * (33 * (10 + 3 + 0 + 2) + 32 * 3 + 35 * 4)
+    assert per_row == (10 + 3 + 0 + 2) / 4
+    ops, per_row = bench._kmeans_ops(16, 10, [])
+    assert ops == 0 and per_row == 0
