@@ -698,6 +698,65 @@ __global__ void __launch_bounds__(256) kmeans_bag_half_kernel(const __grid_const
     }
 }
 
+// d <= 16: each half-warp walks its own bags (lane c of the half: element c and centroid c),
+// so a warp has two bags in flight; the halves' shuffles name only their own 16 lanes.
+__global__ void __launch_bounds__(256) kmeans_bag16_kernel(const __grid_constant__ KmeansBagTables tabs,
+                                                           const KmeansBagArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int h = lane >> 4, c = lane & 15;
+    const unsigned hmask = 0xffffu << (16 * h);
+    const int64_t half = (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5) * 2 + h;
+    const int64_t halves = (((int64_t)gridDim.x * blockDim.x) >> 5) * 2;
+    const int64_t G = (int64_t)a.T * a.batch;
+    const int32_t total = __ldg(a.offsets + G);
+    int32_t np0 = 0, np1 = 0, nid = -1;
+    if (half < G) {
+        np0 = __ldg(a.offsets + half);
+        np1 = __ldg(a.offsets + half + 1);
+        nid = half < total ? __ldg(a.indices + half) : -1;
+    }
+    for (int64_t g = half; g < G; g += halves) {
+        int32_t p0 = np0, p1 = np1;
+        const int32_t own = nid;
+        const int64_t gn = g + halves;
+        if (gn < G) {
+            np0 = __ldg(a.offsets + gn);
+            np1 = __ldg(a.offsets + gn + 1);
+            nid = gn < total ? __ldg(a.indices + gn) : -1;
+        }
+        const int t = (int)div_batch((uint32_t)g, a.div);
+        const int64_t b = g - (int64_t)t * a.batch;
+        p0 = p0 < 0 ? 0 : (p0 > total ? total : p0);
+        p1 = p1 < 0 ? 0 : (p1 > total ? total : p1);
+        if (p1 < p0) {
+            if (c == 0)
+                raise_flag(a.flags, DQ_FLAG_BAD_OFFSETS);
+            p1 = p0;
+        }
+        const int64_t n_rows = tabs.n_rows[t];
+        const uint16_t *cbt = tabs.codebook[t];
+        const uint8_t *ct = tabs.codes[t];
+        const int64_t cld = tabs.codes_ld[t];
+        float acc = 0.0f;
+        for (int32_t p = p0; p < p1; ++p) {
+            const int32_t id = (int64_t)p == g ? own : __ldg(a.indices + p);
+            if (id < 0 || id >= n_rows) {
+                if (c == 0)
+                    raise_flag(a.flags, DQ_FLAG_BAD_INDEX);
+                continue;
+            }
+            const float cj = __half2float(__ushort_as_half(__ldg(cbt + 16 * (int64_t)id + c)));
+            unsigned qk = 0;
+            if (c < a.d)
+                qk = (__ldg(ct + (int64_t)id * cld + c / 2) >> (4 * (c & 1))) & 15u;
+            acc = __fadd_rn(acc, __shfl_sync(hmask, cj, (int)qk, 16));
+        }
+        if (c < a.d)
+            a.out[b * (int64_t)a.T * a.d + (int64_t)t * a.d + c] = acc;
+    }
+}
+
 // Calls of many bags at d <= 64: the id count (the last offset) picks the layout, 32 bags
 // per warp when the bags hold under two ids on average, else one warp per bag. (A kernel
 // of its own: the tile layout's registers would cost the smaller calls occupancy.)
@@ -772,6 +831,11 @@ cudaError_t launch_kmeans_bag(const KmeansBagTables &tabs, const KmeansBagArgs &
             kmeans_bag_half_kernel<8><<<grid, 256, 0, stream>>>(tabs, a);
         else
             kmeans_bag_half_kernel<16><<<grid, 256, 0, stream>>>(tabs, a);
+        return cudaGetLastError();
+    }
+    if (a.d <= 16) {
+        const int64_t need16 = (G * 16 + 255) / 256;
+        kmeans_bag16_kernel<<<(unsigned)(need16 < cap ? need16 : cap), 256, 0, stream>>>(tabs, a);
         return cudaGetLastError();
     }
     if (chunks <= 1)

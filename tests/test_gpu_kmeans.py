@@ -182,7 +182,8 @@ def _kmeans_tables(rows, d, seed):
 
 
 @pytest.mark.parametrize("d,pool", [(16, (1, 1)), (16, (0, 10)), (64, (20, 80)), (128, (1, 1)), (37, (0, 5)),
-                                    (256, (3, 9)), (512, (0, 3)), (1024, (1, 1)), (1000, (1, 4)), (64, (0, 2))])
+                                    (256, (3, 9)), (512, (0, 3)), (1024, (1, 1)), (1000, (1, 4)), (64, (0, 2)),
+                                    (5, (0, 3)), (1, (1, 1))])
 def test_kmeans_bag(cuda_device, d, pool):
     rows = [500, 0, 1300] if pool != (1, 1) else [800, 1200]
     T, B = len(rows), 300
