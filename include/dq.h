@@ -40,6 +40,11 @@
  *   - Arguments are validated on the host before anything is enqueued:
  *     DQ_ERR_INVALID_ARG, nothing launched. A failed launch returns DQ_ERR_CUDA.
  *     dq_last_error() gives the calling thread's last detailed message.
+ *   - Typed arrays must be aligned to their element size: binary16 arrays
+ *     (scale_bias, codebook) to 2 bytes, int32 and binary32 arrays (indices,
+ *     offsets, x, out, dest, grad_out, row_loss) to 4 bytes; a misaligned one is
+ *     rejected with DQ_ERR_INVALID_ARG. Byte arrays (codes) have no rule; aligned
+ *     code rows (16-byte rows and codes_ld) take the vectorised kernels.
  *   - n_rows == 0 or batch == 0 is a no-op returning DQ_OK.
  *   - Data errors are preconditions and are never trapped on the device. When
  *     `d_flags` (a device uint32) is non-NULL the kernels OR DQ_FLAG_* bits into

@@ -100,6 +100,9 @@ dq_status dq_quantize_rows_int4(const float *x, int64_t n_rows, int32_t d, int64
         return fail(DQ_ERR_INVALID_ARG, "mode = %d is neither DQ_MODE_GREEDY nor DQ_MODE_MINMAX", mode);
     if (n_rows > 0 && (!x || !codes || !scale_bias))
         return fail(DQ_ERR_INVALID_ARG, "x, codes and scale_bias must be non-NULL when n_rows > 0");
+    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(scale_bias) & 1) ||
+                       (reinterpret_cast<uintptr_t>(row_loss) & 3)))
+        return fail(DQ_ERR_INVALID_ARG, "x and row_loss must be 4-byte and scale_bias 2-byte aligned");
     if (n_rows > ((int64_t)1 << 40))
         return fail(DQ_ERR_INVALID_ARG, "n_rows = %lld beyond 2^40", (long long)n_rows);
     if (n_rows == 0)
@@ -127,6 +130,8 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
         return fail(DQ_ERR_INVALID_ARG, "out_ld = %lld < d = %d", (long long)out_ld, d);
     if (n_rows > 0 && (!codes || !scale_bias || !out))
         return fail(DQ_ERR_INVALID_ARG, "codes, scale_bias and out must be non-NULL when n_rows > 0");
+    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(scale_bias) & 1) || (reinterpret_cast<uintptr_t>(out) & 3)))
+        return fail(DQ_ERR_INVALID_ARG, "scale_bias must be 2-byte and out 4-byte aligned");
     if (n_rows == 0)
         return ok();
     int sms = 0;
@@ -140,6 +145,9 @@ dq_status dq_dequantize_rows(const uint8_t *codes, int64_t codes_ld, const uint1
 }
 
 namespace {
+
+// Element alignment of a typed array (a misaligned one would fault in the kernels).
+bool misaligned(const void *p, uintptr_t bytes) { return (reinterpret_cast<uintptr_t>(p) & (bytes - 1)) != 0; }
 
 // Checks and copies the lookup's tables (column block t of each output row by default).
 dq_status bag_tables(const dq_table *tables, int32_t n_tables, int32_t d, int32_t batch, dq::BagTables &tabs)
@@ -164,6 +172,8 @@ dq_status bag_tables(const dq_table *tables, int32_t n_tables, int32_t d, int32_
                         (long long)tb.codes_ld, (d + 1) / 2);
         if (tb.n_rows > 0 && (!tb.codes || !tb.scale_bias))
             return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codes and scale_bias must be non-NULL", t);
+        if (tb.n_rows > 0 && misaligned(tb.scale_bias, 2))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: scale_bias must be 2-byte aligned", t);
         tabs.codes[t] = tb.codes;
         tabs.scale_bias[t] = tb.scale_bias;
         tabs.n_rows[t] = tb.n_rows;
@@ -196,6 +206,8 @@ dq_status dq_embbag_int4_fwd(const dq_table *tables, int32_t n_tables, int32_t d
         return st;
     if (batch > 0 && (!indices || !offsets || !out))
         return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
+    if (batch > 0 && (misaligned(indices, 4) || misaligned(offsets, 4) || misaligned(out, 4)))
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be 4-byte aligned");
     if (batch == 0)
         return ok();
     dq::BagArgs a{};
@@ -242,10 +254,14 @@ dq_status dq_embbag_int4_fwd_to_owners(const dq_table *tables, int32_t n_tables,
         return fail(DQ_ERR_INVALID_ARG, "the destination buffers exceed 2^40 elements");
     if (batch > 0 && (!indices || !offsets))
         return fail(DQ_ERR_INVALID_ARG, "indices and offsets must be non-NULL when batch > 0");
+    if (batch > 0 && (misaligned(indices, 4) || misaligned(offsets, 4)))
+        return fail(DQ_ERR_INVALID_ARG, "indices and offsets must be 4-byte aligned");
     dq::BagDest dst{};
     for (int r = 0; r < n_dest; ++r) {
         if (batch > 0 && !dest[r])
             return fail(DQ_ERR_INVALID_ARG, "dest[%d] must be non-NULL", r);
+        if (batch > 0 && misaligned(dest[r], 4))
+            return fail(DQ_ERR_INVALID_ARG, "dest[%d] must be 4-byte aligned", r);
         dst.ptr[r] = dest[r];
     }
     if (batch == 0)
@@ -310,8 +326,9 @@ dq_status dq_quantize_rows_kmeans4(const float *x, int64_t n_rows, int32_t d, in
         return fail(DQ_ERR_INVALID_ARG, "iters = %d outside [0, %d]", iters, DQ_KMEANS_MAX_ITERS);
     if (n_rows > 0 && (!x || !codes || !codebook))
         return fail(DQ_ERR_INVALID_ARG, "x, codes and codebook must be non-NULL when n_rows > 0");
-    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(codebook) & 1)))
-        return fail(DQ_ERR_INVALID_ARG, "x must be 4-byte and codebook 2-byte aligned");
+    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(x) & 3) || (reinterpret_cast<uintptr_t>(codebook) & 1) ||
+                       (reinterpret_cast<uintptr_t>(row_loss) & 3) || (reinterpret_cast<uintptr_t>(row_iters) & 3)))
+        return fail(DQ_ERR_INVALID_ARG, "x, row_loss and row_iters must be 4-byte and codebook 2-byte aligned");
     if (n_rows == 0)
         return ok();
     int sms = 0;
@@ -337,6 +354,8 @@ dq_status dq_dequantize_rows_kmeans4(const uint8_t *codes, int64_t codes_ld, con
         return fail(DQ_ERR_INVALID_ARG, "out_ld = %lld < d = %d", (long long)out_ld, d);
     if (n_rows > 0 && (!codes || !codebook || !out))
         return fail(DQ_ERR_INVALID_ARG, "codes, codebook and out must be non-NULL when n_rows > 0");
+    if (n_rows > 0 && ((reinterpret_cast<uintptr_t>(codebook) & 1) || (reinterpret_cast<uintptr_t>(out) & 3)))
+        return fail(DQ_ERR_INVALID_ARG, "codebook must be 2-byte and out 4-byte aligned");
     if (n_rows == 0)
         return ok();
     int sms = 0;
@@ -374,6 +393,8 @@ dq_status dq_embbag_kmeans4_fwd(const dq_kmeans_table *tables, int32_t n_tables,
                         (long long)tb.codes_ld, (d + 1) / 2);
         if (tb.n_rows > 0 && (!tb.codes || !tb.codebook))
             return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codes and codebook must be non-NULL", t);
+        if (tb.n_rows > 0 && misaligned(tb.codebook, 2))
+            return fail(DQ_ERR_INVALID_ARG, "tables[%d]: codebook must be 2-byte aligned", t);
         tabs.codes[t] = tb.codes;
         tabs.codebook[t] = tb.codebook;
         tabs.n_rows[t] = tb.n_rows;
@@ -381,6 +402,8 @@ dq_status dq_embbag_kmeans4_fwd(const dq_kmeans_table *tables, int32_t n_tables,
     }
     if (batch > 0 && (!indices || !offsets || !out))
         return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be non-NULL when batch > 0");
+    if (batch > 0 && (misaligned(indices, 4) || misaligned(offsets, 4) || misaligned(out, 4)))
+        return fail(DQ_ERR_INVALID_ARG, "indices, offsets and out must be 4-byte aligned");
     if (batch == 0)
         return ok();
     int sms = 0;

@@ -206,3 +206,49 @@ def test_kmeans_dequantize_and_bag_reject(L):
     arr0 = (dq._KmeansTable * 1)(dq._KmeansTable(None, None, 0, 8))
     assert L.dq_embbag_kmeans4_fwd(ctypes.cast(arr0, ctypes.c_void_p), 1, 16, None, None, 0, None, None,
                                    None) == dq.DQ_OK
+
+
+def test_misaligned_arrays_are_rejected_before_any_launch(L):
+    """Typed arrays the kernels read element-wise must be aligned to their element size."""
+    A = 1 << 24   # stand-in device addresses: only compared and checked, never touched
+    # dequantize: binary16 scale/bias, binary32 output
+    assert L.dq_dequantize_rows(A, 8, A + 1, 3, 16, A, 16, None) == dq.DQ_ERR_INVALID_ARG
+    assert "2-byte" in L.dq_last_error().decode()
+    assert L.dq_dequantize_rows(A, 8, A, 3, 16, A + 2, 16, None) == dq.DQ_ERR_INVALID_ARG
+    assert "4-byte" in L.dq_last_error().decode()
+    assert L.dq_dequantize_rows_kmeans4(A, 8, A + 1, 3, 16, A, 16, None) == dq.DQ_ERR_INVALID_ARG
+    assert "2-byte" in L.dq_last_error().decode()
+    # lookup: a table's scale/bias, the ids, offsets and output
+    p, keep = _tables((A, A + 1, 10, 8))
+    assert L.dq_embbag_int4_fwd(p, 1, 16, A, A, 4, A, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "scale_bias must be 2-byte" in L.dq_last_error().decode()
+    p, keep = _tables((A, A, 10, 8))
+    for idx, off, out in ((A + 2, A, A), (A, A + 1, A), (A, A, A + 2)):
+        assert L.dq_embbag_int4_fwd(p, 1, 16, idx, off, 4, out, None, None) == dq.DQ_ERR_INVALID_ARG
+        assert "4-byte aligned" in L.dq_last_error().decode()
+    # the owners' buffers
+    sl = (ctypes.c_int32 * 1)(0)
+    dest = (ctypes.c_void_p * 2)(A, A + 2)
+    assert L.dq_embbag_int4_fwd_to_owners(p, 1, 16, A, A, 4, ctypes.cast(sl, ctypes.c_void_p), 1,
+                                          ctypes.cast(dest, ctypes.c_void_p), 2, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "dest[1] must be 4-byte" in L.dq_last_error().decode()
+    # codebook tables
+    arr = (dq._KmeansTable * 1)(dq._KmeansTable(A, A + 1, 10, 8))
+    assert L.dq_embbag_kmeans4_fwd(ctypes.cast(arr, ctypes.c_void_p), 1, 16, A, A, 4, A, None,
+                                   None) == dq.DQ_ERR_INVALID_ARG
+    assert "codebook must be 2-byte" in L.dq_last_error().decode()
+    arr = (dq._KmeansTable * 1)(dq._KmeansTable(A, A, 10, 8))
+    assert L.dq_embbag_kmeans4_fwd(ctypes.cast(arr, ctypes.c_void_p), 1, 16, A + 2, A, 4, A, None,
+                                   None) == dq.DQ_ERR_INVALID_ARG
+    assert "4-byte aligned" in L.dq_last_error().decode()
+
+
+def test_quantizer_outputs_must_be_aligned(L):
+    A = 1 << 24
+    assert L.dq_quantize_rows_int4(A + 2, 4, 16, 16, A, 8, A, None, None, 0, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "4-byte" in L.dq_last_error().decode()
+    assert L.dq_quantize_rows_int4(A, 4, 16, 16, A, 8, A + 1, None, None, 0, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "scale_bias 2-byte" in L.dq_last_error().decode()
+    assert L.dq_quantize_rows_int4(A, 4, 16, 16, A, 8, A, A + 2, None, 0, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert L.dq_quantize_rows_kmeans4(A, 4, 16, 16, A, 8, A, None, A + 1, 10, None, None) == dq.DQ_ERR_INVALID_ARG
+    assert "row_iters" in L.dq_last_error().decode()
