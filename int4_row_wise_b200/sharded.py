@@ -52,6 +52,27 @@ def _check_owner(owner: Sequence[int], world: int) -> None:
         raise ValueError(f"owner ranks {bad[:4]} outside [0, {world})")
 
 
+def _agree(err: Optional[str], group, device) -> None:
+    """Every rank learns, before any exchange, whether some rank's arguments failed its
+    checks (one all-reduce of a flag), and then all of them raise: a rank with bad
+    arguments cannot leave the others waiting in an exchange it never joins. Also a
+    barrier: it returns once every rank has reached it."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_initialized() or dist.get_world_size(group) == 1:
+        if err:
+            raise ValueError(err)
+        return
+    if dist.get_backend(group) != "nccl":
+        device = torch.device("cpu")
+    flag = torch.tensor([1 if err else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(flag, op=dist.ReduceOp.MAX, group=group)
+    if err:
+        raise ValueError(err)
+    if int(flag.item()):
+        raise ValueError("another rank's arguments failed their checks")
+
+
 def _reassemble(recv, owner: Sequence[int], world: int, bl: int, d: int):
     """[bl, T * d] in global table order from the received buffer, which holds, source
     by source, [bl, tables of that source, d]. One concatenation kernel."""
@@ -74,7 +95,7 @@ def _reassemble(recv, owner: Sequence[int], world: int, bl: int, d: int):
 
 
 def sharded_embbag(local_tables: Sequence, owner: Sequence[int], d: int, indices, offsets, global_batch: int,
-                   group=None, lookup: Optional[Callable] = None):
+                   group=None, lookup: Optional[Callable] = None, _checked: bool = False):
     """Pooled outputs of this rank's slice of the global batch, over all tables.
 
     local_tables  the tables this rank owns, in ascending global table order
@@ -85,21 +106,28 @@ def sharded_embbag(local_tables: Sequence, owner: Sequence[int], d: int, indices
     global_batch  bags per table, divisible by the world size
     lookup        (tables, d, indices, offsets, batch) -> [batch, len(tables) * d];
                   dq.embbag by default
-    Returns a [global_batch // world, T * d] tensor on the tables' device."""
+    Returns a [global_batch // world, T * d] tensor on the tables' device. The argument
+    checks are collective: if any rank's fail, every rank raises ValueError."""
     import torch
     import torch.distributed as dist
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    _check_owner(owner, world)
-    if global_batch % world:
-        raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
     mine = [t for t, r in enumerate(owner) if r == rank]
-    if len(mine) != len(local_tables):
-        raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
-    if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
-        raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x {global_batch} bags "
-                         f"need {len(mine) * global_batch + 1}")
+    if not _checked:
+        err = None
+        try:
+            _check_owner(owner, world)
+            if global_batch % world:
+                raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
+            if len(mine) != len(local_tables):
+                raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
+            if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
+                raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x "
+                                 f"{global_batch} bags need {len(mine) * global_batch + 1}")
+        except ValueError as e:
+            err = str(e)
+        _agree(err, group, offsets.device)
     if lookup is None:
         import int4_row_wise_b200 as dq
         lookup = dq.embbag
@@ -135,14 +163,22 @@ def sharded_embbag_local(local_tables: Sequence, owner: Sequence[int], d: int, b
 
     world = dist.get_world_size(group)
     rank = dist.get_rank(group)
-    _check_owner(owner, world)
     T = len(owner)
-    if len(batches) != T:
-        raise ValueError(f"{len(batches)} batches for {T} tables")
-    for t, (_, off) in enumerate(batches):
-        if int(off.numel()) != local_batch + 1:
-            raise ValueError(f"table {t}: offsets hold {int(off.numel())} entries, local_batch + 1 = "
-                             f"{local_batch + 1} expected")
+    err = None
+    try:
+        _check_owner(owner, world)
+        if len(batches) != T:
+            raise ValueError(f"{len(batches)} batches for {T} tables")
+        for t, (_, off) in enumerate(batches):
+            if int(off.numel()) != local_batch + 1:
+                raise ValueError(f"table {t}: offsets hold {int(off.numel())} entries, local_batch + 1 = "
+                                 f"{local_batch + 1} expected")
+        mine_n = sum(1 for r in owner if r == rank)
+        if mine_n != len(local_tables):
+            raise ValueError(f"rank {rank} owns {mine_n} tables by the plan but holds {len(local_tables)}")
+    except ValueError as e:
+        err = str(e)
+    _agree(err, group, batches[0][1].device if batches else torch.device("cpu"))
     dev = batches[0][1].device
     to = [[t for t in range(T) if owner[t] == s] for s in range(world)]
     mine = to[rank]
@@ -185,7 +221,7 @@ def sharded_embbag_local(local_tables: Sequence, owner: Sequence[int], d: int, b
     offsets = torch.zeros(len(mine) * world * local_batch + 1, dtype=torch.int32, device=dev)
     offsets[1:] = torch.cumsum(lens.permute(1, 0, 2).reshape(-1), dim=0).to(torch.int32)
     return sharded_embbag(local_tables, owner, d, indices, offsets, world * local_batch, group=group,
-                          lookup=lookup)
+                          lookup=lookup, _checked=True)
 
 
 class OwnerBuffers:
@@ -235,24 +271,28 @@ def sharded_embbag_direct(local_tables: Sequence, owner: Sequence[int], d: int, 
 
     world = dist.get_world_size(group) if dist.is_initialized() else 1
     rank = dist.get_rank(group) if dist.is_initialized() else 0
-    _check_owner(owner, world)
-    if global_batch % world:
-        raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
-    if len(buffers.addresses) != world:
-        raise ValueError(f"{len(buffers.addresses)} owner buffers for {world} ranks")
     T = len(owner)
-    if tuple(buffers.own.shape) != (global_batch // world, T * d):
-        raise ValueError(f"own buffer {tuple(buffers.own.shape)}, expected {(global_batch // world, T * d)}")
     mine = [t for t, r in enumerate(owner) if r == rank]
-    if len(mine) != len(local_tables):
-        raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
-    if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
-        raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x {global_batch} bags "
-                         f"need {len(mine) * global_batch + 1}")
+    err = None
+    try:
+        _check_owner(owner, world)
+        if global_batch % world:
+            raise ValueError(f"global batch {global_batch} is not divisible by the world size {world}")
+        if len(buffers.addresses) != world:
+            raise ValueError(f"{len(buffers.addresses)} owner buffers for {world} ranks")
+        if tuple(buffers.own.shape) != (global_batch // world, T * d):
+            raise ValueError(f"own buffer {tuple(buffers.own.shape)}, expected {(global_batch // world, T * d)}")
+        if len(mine) != len(local_tables):
+            raise ValueError(f"rank {rank} owns {len(mine)} tables by the plan but holds {len(local_tables)}")
+        if mine and int(offsets.numel()) != len(mine) * global_batch + 1:
+            raise ValueError(f"offsets hold {int(offsets.numel())} entries; {len(mine)} tables x {global_batch} "
+                             f"bags need {len(mine) * global_batch + 1}")
+    except ValueError as e:
+        err = str(e)
+    if world > 1:   # the owners have read the previous result (the agreement is the barrier)
+        torch.cuda.current_stream(buffers.own.device).synchronize()
+    _agree(err, group, buffers.own.device)
     stream = torch.cuda.current_stream(buffers.own.device)
-    if world > 1:   # the owners have read the previous result
-        stream.synchronize()
-        dist.barrier(group)
     if mine:
         dq.dq_embbag_int4_fwd_to_owners(local_tables, d, indices, offsets, global_batch, mine, T,
                                         buffers.addresses, None, stream)

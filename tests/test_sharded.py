@@ -236,3 +236,47 @@ def test_routed_lookup_from_local_batches(world, T, bl, seed):
         idx, off = _batch_of(list(range(T)), batches)
         want = _oracle_lookup(tables, D, torch.from_numpy(idx), torch.from_numpy(off), bl).numpy()
         assert np.array_equal(results[r].view(np.uint32), want.view(np.uint32)), r
+
+
+def _rank_bad_args(rank, world, port, which, results):
+    import datetime
+    from int4_row_wise_b200.sharded import sharded_embbag_local
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    # a short timeout: were the checks not collective, the good rank would wait in the
+    # exchange until it ran out, and fail with a timeout instead of a ValueError
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        T, B = 4, 6
+        rows, tables, per_table = _problem(T, B, 7)
+        owner = plan_tables(rows, world)
+        mine = [t for t in range(T) if owner[t] == rank]
+        idx, off = _batch_of(mine, per_table)
+        ti, to = torch.from_numpy(idx), torch.from_numpy(off)
+        try:
+            if which == "global":
+                if rank == world - 1:
+                    to = to[:-1]   # this rank's offsets are one short
+                sharded_embbag([tables[t] for t in mine], owner, D, ti, to, B, lookup=_oracle_lookup)
+            else:
+                bt = [(torch.from_numpy(i), torch.from_numpy(o)) for i, o in per_table]
+                lb = B if rank != world - 1 else B - 1   # this rank's batch size disagrees with its offsets
+                sharded_embbag_local([tables[t] for t in mine], owner, D, bt, lb, lookup=_oracle_lookup)
+            results[rank] = "no error"
+        except ValueError as e:
+            results[rank] = "ValueError: " + str(e)
+        except Exception as e:   # e.g. a collective that timed out
+            results[rank] = type(e).__name__ + ": " + str(e)[:200]
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("which", ["global", "local"])
+def test_bad_arguments_on_one_rank_fail_every_rank(which):
+    world = 2
+    mgr = mp.get_context("spawn").Manager()
+    results = mgr.dict()
+    mp.start_processes(_rank_bad_args, args=(world, _free_port(), which, results), nprocs=world,
+                       start_method="spawn")
+    assert results[world - 1].startswith("ValueError: ") and "another rank" not in results[world - 1], results
+    assert results[0] == "ValueError: another rank's arguments failed their checks", results
