@@ -146,6 +146,26 @@ def test_bag_to_owners_matches_oracle(cuda_device, n_dest, d, pool):
     assert np.array_equal(got[one].view(np.uint32), ref[one].view(np.uint32))
 
 
+@pytest.mark.parametrize("d", [16, 64, 100])
+def test_bag_to_owners_flags_bad_ids(cuda_device, d):
+    """Invalid ids are skipped and flagged in the owner-store form as in the plain lookup."""
+    T, B = 2, 64
+    rows = [300, 40]
+    cld = ((d + 1) // 2 + 15) // 16 * 16
+    tabs = [_packed(n, d, 70 + t, cld) for t, n in enumerate(rows)]
+    idx, off = _bags(T, B, rows, 1, 6, d, bad=True)
+    ref, mag, skipped = oracle.embbag(tabs, d, idx, off, B, with_abs_sum=True)
+    assert skipped > 0
+    dest = [torch.zeros((B // 2, T * d), dtype=torch.float32, device="cuda") for _ in range(2)]
+    fl = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dev_tabs = [dq.PackedTable(to_dev(c), to_dev(s.view(np.int16))) for c, s in tabs]
+    dq.dq_embbag_int4_fwd_to_owners(dev_tabs, d, to_dev(idx), to_dev(off), B, [0, 1], T, dest, d_flags=fl)
+    torch.cuda.synchronize()
+    got = np.concatenate([x.cpu().numpy() for x in dest])
+    bag_tolerance_check(got, ref, mag)
+    assert fl.item() & dq.DQ_FLAG_BAD_INDEX
+
+
 def test_bag_bad_ids_and_offsets(cuda_device):
     d, T, B = 64, 2, 50
     rows = [100, 100]
